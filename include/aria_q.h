@@ -1,0 +1,156 @@
+/*
+ * aria_q.h -- C ABI of libaria_q.so: quantized linear layers (q8 / q4
+ * weight-only, W8A8) for NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "A Quantized Native Runtime for On-Device Semantic
+ * Audio Generation" (aria project page). "What aria is": the diffusion
+ * transformer's weights are packed from fp16 to 8 or 4 bits and the fp16
+ * copy is released, so the packed form replaces the footprint. "Results":
+ * four precisions -- fp16, q8, W8A8 (8-bit arithmetic on integer tensor
+ * cores, the fastest GPU mode) and q4; q8 and W8A8 share one footprint.
+ * "Steering is real": a direction vector is added at one transformer block,
+ * and alpha = 0 removes it with bit-identical output.
+ *
+ * Formats (the pages give none; these are the library's fixed readings):
+ *   Q8 / W8A8 weights: Wq int8 [N,K] row-major (K contiguous),
+ *       scales fp32 [N]; s[n] = absmax_k|W[n,k]| / 127 (fp32 division),
+ *       Wq = clamp(round_half_even(W / s), -127, 127); all-zero row -> s = 0.
+ *   Q4 weights (group 32 along K): Wq uint8 [N,K/2]; byte k/2 holds k even in
+ *       its low nibble and k odd in its high nibble, each as code+8 (offset
+ *       binary); scales fp16 [N,K/32]; s16 = fp16_rn(absmax/7),
+ *       code = clamp(round_half_even(W / float(s16)), -7, 7).
+ *   Activations for W8A8: Xq int8 [M,K], s_x fp32 [M], the Q8 rule per token row.
+ *   X, W, bias, Y: fp16 (IEEE binary16), row-major; Y is [M,N].
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are caller-owned device memory on the current
+ *     CUDA device; the library keeps no pointer after the call returns.
+ *   - Every device pointer must be 16-byte aligned (ARIA_ERR_MISALIGNED).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *     enqueued on it; calls return after launch, without synchronising.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns an error and launches nothing.
+ *   - Kernels bound every wait. A wait that runs out (about 4 s) records
+ *     ARIA_ERR_TIMEOUT in a device status word, and the kernel returns;
+ *     aria_device_status() reports and clears it.
+ *   - Non-finite inputs are outside the contract (not checked).
+ *   - The library allocates no device memory, makes no host-device copies
+ *     inside the entry points below, and is safe to call while a stream is
+ *     being captured into a CUDA graph (aria_device_status excepted).
+ */
+#ifndef ARIA_Q_H
+#define ARIA_Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ARIA_OK = 0,
+    ARIA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive or too-large size */
+    ARIA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (group != 32, shape rule) */
+    ARIA_ERR_MISALIGNED = 3,   /* a device pointer is not 16-byte aligned */
+    ARIA_ERR_CUDA = 4,         /* a CUDA runtime call failed (see aria_last_error_message) */
+    ARIA_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (device status word) */
+} aria_status;
+
+typedef enum {
+    ARIA_FMT_Q8 = 1,    /* 8-bit weights, fp16 activations (weight-only) */
+    ARIA_FMT_Q4 = 2,    /* 4-bit group-32 weights, fp16 activations (weight-only) */
+    ARIA_FMT_W8A8 = 3   /* 8-bit weights (the Q8 pack) x per-token int8 activations */
+} aria_format;
+
+/* Human-readable name of a status code (static string). */
+const char *aria_status_string(aria_status s);
+
+/* Text of the last error returned on the calling host thread ("" if none). */
+const char *aria_last_error_message(void);
+
+/*
+ * aria_qpack_size -- bytes of the packed weights and of their scales.
+ * ("What aria is": weights packed from fp16 to 8 or 4 bits.)
+ *   fmt    ARIA_FMT_Q8 or ARIA_FMT_W8A8 (same pack), or ARIA_FMT_Q4.
+ *   group  0 for Q8 / W8A8 (per output channel); 32 for Q4.
+ *   N, K   output and input features of the linear layer (W is [N,K]).
+ *   wq_bytes, scale_bytes  host outputs: N*K and 4*N (Q8), N*K/2 and 2*N*K/32 (Q4).
+ * Errors: INVALID_ARG (NULL outputs, N or K <= 0), UNSUPPORTED (group, K % 32 for Q4).
+ */
+aria_status aria_qpack_size(aria_format fmt, int group, int64_t N, int64_t K,
+                            size_t *wq_bytes, size_t *scale_bytes);
+
+/*
+ * aria_qpack -- pack fp16 weights W [N,K] into the Q8 or Q4 format above.
+ * ("What aria is": the fp16 copy is released once packed -- the caller may
+ * free W after the stream reaches this call; the library never holds it.)
+ *   W       device, fp16 [N,K] row-major.
+ *   Wq      device output, int8 [N,K] (Q8, W8A8) or uint8 [N,K/2] (Q4).
+ *   scales  device output, fp32 [N] (Q8, W8A8) or fp16 [N,K/32] (Q4).
+ * Shape rules: N >= 1; K >= 16 and K % 16 == 0 (Q8); K % 32 == 0 (Q4).
+ * Packed bytes are a pure function of W (bit-exact, deterministic).
+ */
+aria_status aria_qpack(aria_format fmt, int group, const void *W, int64_t N, int64_t K,
+                       void *Wq, void *scales, void *stream);
+
+/*
+ * aria_act_quant -- per-token dynamic int8 quantisation of activations (the
+ * "A8" of W8A8, "Results": 8-bit arithmetic on integer tensor cores).
+ *   X   device, fp16 [M,K] row-major.
+ *   Xq  device output, int8 [M,K]; sx device output, fp32 [M].
+ *   s_x[m] = absmax_k |X[m,k]| / 127; Xq = clamp(rhe(X / s_x[m]), -127, 127).
+ * Shape rules: M >= 1, K >= 16, K % 16 == 0. Bit-exact and deterministic.
+ */
+aria_status aria_act_quant(const void *X, int64_t M, int64_t K, int8_t *Xq, float *sx,
+                           void *stream);
+
+/*
+ * aria_qgemm -- Y = X . dequant(W)^T with the fused epilogue
+ *   Y[m,n] = fp16( main[m,n] + bias[n] + alpha * v[n] ).
+ *   Q8:   main = s_w[n] * sum_k X[m,k] * Wq[n,k]            (fp16 tensor cores)
+ *   Q4:   main = sum_k X[m,k] * fp16((code-8) * s16[n,k/32]) (fp16 tensor cores)
+ *   W8A8: main = acc[m,n] * s_x[m] * s_w[n], acc = sum_k Xq*Wq exact int32
+ *         (int8 tensor cores); the epilogue is evaluated in fp64 and rounded
+ *         once to fp16.
+ *   X       device: fp16 [M,K] (Q8, Q4) or int8 [M,K] from aria_act_quant (W8A8).
+ *   sx      device fp32 [M] (W8A8 only; must be NULL otherwise).
+ *   Wq, scales  device, as produced by aria_qpack (W8A8 takes the Q8 pack).
+ *   bias    device fp16 [N], or NULL for none.
+ *   steer_vec device fp32 [N], or NULL. The steering add ("Steering is real")
+ *           is skipped entirely when steer_vec == NULL or alpha == 0, so the
+ *           output is then bit-identical to an unsteered call.
+ *   Y       device output, fp16 [M,N] row-major. Must not alias any input.
+ * Shape rules: M >= 1; N >= 16, N % 16 == 0; K >= 16, K % 16 == 0;
+ *   Q4 additionally K % 256 == 0; group as in aria_qpack_size.
+ * Deterministic: the same inputs give the same bytes on every call.
+ */
+aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
+                       const void *X, const float *sx, const void *Wq, const void *scales,
+                       const void *bias, const float *steer_vec, float alpha, void *Y,
+                       void *stream);
+
+/*
+ * aria_qgemm_s32 -- the W8A8 integer GEMM alone: C[m,n] = sum_k Xq[m,k]*Wq[n,k]
+ * as exact int32 ("Results": 8-bit arithmetic on integer tensor cores). Runs
+ * the same tensor-core mainloop as aria_qgemm(ARIA_FMT_W8A8) and stores the
+ * raw accumulators, for bit-exact checks.
+ *   Xq device int8 [M,K]; Wq device int8 [N,K]; C device output int32 [M,N].
+ * Shape rules as for aria_qgemm. The caller keeps K * 127^2 < 2^31.
+ */
+aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t *Xq, const int8_t *Wq,
+                           int32_t *C, void *stream);
+
+/*
+ * aria_device_status -- synchronise `stream`, then read and clear the device
+ * status word of the current device. Returns ARIA_ERR_TIMEOUT if any kernel
+ * of this library gave up on a bounded wait since the last call, ARIA_ERR_CUDA
+ * if the stream reports an error, else ARIA_OK. Not for use during capture.
+ */
+aria_status aria_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARIA_Q_H */

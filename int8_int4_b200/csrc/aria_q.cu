@@ -1,0 +1,387 @@
+// aria_q.cu -- the C ABI of libaria_q.so (declared in include/aria_q.h):
+// host-side validation, tensor-map encoding, tile / split planning and
+// launches of the sm_100a kernels. One translation unit, so the device
+// status word is a single symbol without relocatable device code.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "aria_q.h"
+#include "ptx.cuh"
+#include "qgemm.cuh"
+#include "quant_kernels.cuh"
+
+#define ARIA_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+aria_status fail(aria_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+aria_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(ARIA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+
+// ------------------------------------------------------------ tensor maps ---
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements; box {bc, br}.
+aria_status make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
+                     int64_t rows, int64_t cols, int bc, int br, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ARIA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esize)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(bc), static_cast<cuuint32_t>(br)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ARIA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ARIA_OK;
+}
+
+// ---------------------------------------------------------- device facts ---
+struct DevInfo {
+  int sms = 148;
+  int smem_optin = 232448;
+};
+
+DevInfo dev_info() {
+  static DevInfo info[16];
+  static bool done[16] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> g(mu);
+  if (dev >= 0 && dev < 16 && !done[dev]) {
+    cudaDeviceGetAttribute(&info[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&info[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    done[dev] = true;
+  }
+  return (dev >= 0 && dev < 16) ? info[dev] : DevInfo{};
+}
+
+// ----------------------------------------------------------------- GEMM ---
+struct Plan {
+  aria::GemmParams p;
+  dim3 grid;
+  size_t smem;
+};
+
+aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
+  using namespace aria;
+  const DevInfo di = dev_info();
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  const int unitK = kind == kQ4 ? 256 : 128;
+  p.units = static_cast<int>((K + unitK - 1) / unitK);
+
+  int mt = static_cast<int>((M + 255) / 256);
+  int bn = static_cast<int>((M + mt - 1) / mt);
+  bn = (bn + 15) / 16 * 16;
+  mt = static_cast<int>((M + bn - 1) / bn);
+  p.BN = bn;
+  const int nt = static_cast<int>((N + kTileN - 1) / kTileN);
+  const int64_t tiles = static_cast<int64_t>(nt) * mt;
+  if (mt > 65535 || nt > 65535) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
+
+  int splits = 1;
+  if (tiles < di.sms) splits = static_cast<int>(std::min<int64_t>(8, di.sms / tiles));
+  splits = std::max(1, std::min(splits, p.units));
+  p.splits = splits;
+
+  p.x_stage = static_cast<uint32_t>(bn) * 128u;
+  const bool dq = (kind == kQ8 || kind == kQ4);
+  p.raw_stage = kind == kQ8 ? kATile : (kind == kQ4 ? kATile + kQ4ScaleTile : 0);
+  p.raw_stage = (p.raw_stage + 1023u) & ~1023u;
+  const int64_t budget = static_cast<int64_t>(di.smem_optin) - 1024 - 1024;  // align + barriers
+  int nr = 0, na = 0, nx = 0;
+  if (dq) {
+    na = bn > 128 ? 3 : 4;
+    for (int k = 8; k >= 2; --k) {
+      const int64_t need = static_cast<int64_t>(k) * p.raw_stage + na * kATile + k * p.x_stage;
+      if (need <= budget) { nr = nx = k; break; }
+    }
+    if (nr == 0) return fail(ARIA_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  } else {
+    for (int k = 8; k >= 2; --k) {
+      if (static_cast<int64_t>(k) * (kATile + p.x_stage) <= budget) { na = nx = k; break; }
+    }
+    if (na == 0) return fail(ARIA_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  }
+  p.n_raw = nr;
+  p.n_a = na;
+  p.n_x = nx;
+  p.off_raw = 0;
+  p.off_a = p.off_raw + nr * p.raw_stage;
+  p.off_x = p.off_a + na * kATile;
+  p.off_bar = p.off_x + nx * p.x_stage;
+  if (splits > 1 && static_cast<uint32_t>(bn) * 512u > p.off_bar)
+    return fail(ARIA_ERR_UNSUPPORTED, "split-K buffer does not fit");
+  const uint32_t nbar = 2 * (nr + na + nx) + 1;
+  const size_t smem = 1024 + p.off_bar + nbar * 8 + 16;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(bn)) cols <<= 1;
+  p.tmem_cols = cols;
+
+  out->p = p;
+  out->grid = dim3(splits, nt, mt);
+  out->smem = smem;
+  return ARIA_OK;
+}
+
+template <int KIND>
+aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap& ts,
+                        const CUtensorMap& tx, cudaStream_t st) {
+  auto kfn = aria::qgemm_kernel<KIND>;
+  static int configured_for = -1;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    // set once per process and device-independent: the attribute is per function
+    if (configured_for != dev) {
+      cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           dev_info().smem_optin);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      configured_for = dev;
+    }
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = pl.grid;
+  cfg.blockDim = dim3(aria::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = 0;
+  if (pl.p.splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, pl.p);
+  if (e != cudaSuccess) return cuda_fail(e, "qgemm launch");
+  return ARIA_OK;
+}
+
+aria_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+    return fail(ARIA_ERR_INVALID_ARG, "sizes must be positive and < 2^31 (M=%lld N=%lld K=%lld)",
+                (long long)M, (long long)N, (long long)K);
+  if (N < 16 || N % 16) return fail(ARIA_ERR_UNSUPPORTED, "N must be a positive multiple of 16");
+  if (K < 16 || K % 16) return fail(ARIA_ERR_UNSUPPORTED, "K must be a positive multiple of 16");
+  return ARIA_OK;
+}
+
+}  // namespace
+
+// ================================================================= ABI ===
+
+ARIA_API const char* aria_status_string(aria_status s) {
+  switch (s) {
+    case ARIA_OK: return "ARIA_OK";
+    case ARIA_ERR_INVALID_ARG: return "ARIA_ERR_INVALID_ARG";
+    case ARIA_ERR_UNSUPPORTED: return "ARIA_ERR_UNSUPPORTED";
+    case ARIA_ERR_MISALIGNED: return "ARIA_ERR_MISALIGNED";
+    case ARIA_ERR_CUDA: return "ARIA_ERR_CUDA";
+    case ARIA_ERR_TIMEOUT: return "ARIA_ERR_TIMEOUT";
+  }
+  return "ARIA_ERR_UNKNOWN";
+}
+
+ARIA_API const char* aria_last_error_message(void) { return g_msg; }
+
+ARIA_API aria_status aria_qpack_size(aria_format fmt, int group, int64_t N, int64_t K,
+                                     size_t* wq_bytes, size_t* scale_bytes) {
+  if (!wq_bytes || !scale_bytes) return fail(ARIA_ERR_INVALID_ARG, "NULL output pointer");
+  if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim)
+    return fail(ARIA_ERR_INVALID_ARG, "N and K must be in [1, 2^31)");
+  if (fmt == ARIA_FMT_Q8 || fmt == ARIA_FMT_W8A8) {
+    if (group != 0) return fail(ARIA_ERR_UNSUPPORTED, "q8 scales are per output channel: group must be 0");
+    *wq_bytes = static_cast<size_t>(N) * K;
+    *scale_bytes = static_cast<size_t>(N) * 4;
+    return ARIA_OK;
+  }
+  if (fmt == ARIA_FMT_Q4) {
+    if (group != 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 supports group = 32 only");
+    if (K % 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 needs K % 32 == 0");
+    *wq_bytes = static_cast<size_t>(N) * (K / 2);
+    *scale_bytes = static_cast<size_t>(N) * (K / 32) * 2;
+    return ARIA_OK;
+  }
+  return fail(ARIA_ERR_INVALID_ARG, "unknown format %d", (int)fmt);
+}
+
+ARIA_API aria_status aria_qpack(aria_format fmt, int group, const void* W, int64_t N, int64_t K,
+                                void* Wq, void* scales, void* stream) {
+  size_t wb = 0, sb = 0;
+  aria_status s = aria_qpack_size(fmt, group, N, K, &wb, &sb);
+  if (s != ARIA_OK) return s;
+  if (!W || !Wq || !scales) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(scales))
+    return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fmt == ARIA_FMT_Q4) {
+    const int64_t nchunk = N * (K / 8);
+    const int64_t blocks = std::min<int64_t>((nchunk + 255) / 256, 148 * 16);
+    aria::pack_q4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const __half*>(W), nchunk, static_cast<uint32_t*>(Wq), static_cast<__half*>(scales));
+  } else {
+    if (K % 16) return fail(ARIA_ERR_UNSUPPORTED, "q8 needs K % 16 == 0");
+    aria::row_quant_i8_kernel<<<static_cast<unsigned>(N), aria::kRowThreads, 0, st>>>(
+        static_cast<const __half*>(W), static_cast<int>(K), static_cast<int8_t*>(Wq),
+        static_cast<float*>(scales));
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return ARIA_OK;
+}
+
+ARIA_API aria_status aria_act_quant(const void* X, int64_t M, int64_t K, int8_t* Xq, float* sx,
+                                    void* stream) {
+  if (!X || !Xq || !sx) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  if (M < 1 || K < 1 || M > kMaxDim || K > kMaxDim)
+    return fail(ARIA_ERR_INVALID_ARG, "M and K must be in [1, 2^31)");
+  if (K % 16) return fail(ARIA_ERR_UNSUPPORTED, "K must be a multiple of 16");
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(sx))
+    return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  aria::row_quant_i8_kernel<<<static_cast<unsigned>(M), aria::kRowThreads, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half*>(X), static_cast<int>(K), Xq, sx);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
+  return ARIA_OK;
+}
+
+static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const void* X,
+                              const float* sx, const void* Wq, const void* scales,
+                              const void* bias, const float* steer, float alpha, void* Y,
+                              cudaStream_t st) {
+  using namespace aria;
+  aria_status s = check_gemm_shape(M, N, K);
+  if (s != ARIA_OK) return s;
+  if (kind == kQ4 && K % 256) return fail(ARIA_ERR_UNSUPPORTED, "q4 GEMM needs K % 256 == 0");
+  Plan pl;
+  if ((s = plan_gemm(kind, M, N, K, &pl)) != ARIA_OK) return s;
+  CUtensorMap tw, ts, tx;
+  std::memset(&ts, 0, sizeof(ts));
+  const int bn = pl.p.BN;
+  if (kind == kQ4) {
+    if ((s = make_map(&tw, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
+    if ((s = make_map(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, K / 32, 8, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
+  } else {
+    if ((s = make_map(&tw, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
+  }
+  if (kind == kQ8 || kind == kQ4) {
+    if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, 64, bn,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
+  } else {
+    if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, bn,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
+  }
+  pl.p.sw = static_cast<const float*>(kind == kQ4 ? nullptr : scales);
+  pl.p.sx = sx;
+  pl.p.bias = static_cast<const __half*>(bias);
+  pl.p.steer = (steer && alpha != 0.0f) ? steer : nullptr;  // skip, not "+ 0*v"
+  pl.p.alpha = alpha;
+  pl.p.Y = Y;
+  if (!pl.p.steer) pl.p.alpha = 0.0f;
+  switch (kind) {
+    case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, st);
+    case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, st);
+    case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, st);
+    case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, st);
+  }
+  return fail(ARIA_ERR_INVALID_ARG, "unknown kind");
+}
+
+ARIA_API aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
+                                const void* X, const float* sx, const void* Wq, const void* scales,
+                                const void* bias, const float* steer_vec, float alpha, void* Y,
+                                void* stream) {
+  if (!X || !Wq || !scales || !Y) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  int kind = 0;
+  if (fmt == ARIA_FMT_Q8 || fmt == ARIA_FMT_W8A8) {
+    if (group != 0) return fail(ARIA_ERR_UNSUPPORTED, "q8 scales are per output channel: group must be 0");
+    kind = fmt == ARIA_FMT_Q8 ? aria::kQ8 : aria::kW8A8;
+  } else if (fmt == ARIA_FMT_Q4) {
+    if (group != 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 supports group = 32 only");
+    kind = aria::kQ4;
+  } else {
+    return fail(ARIA_ERR_INVALID_ARG, "unknown format %d", (int)fmt);
+  }
+  if (kind == aria::kW8A8 && !sx) return fail(ARIA_ERR_INVALID_ARG, "W8A8 needs sx");
+  if (kind != aria::kW8A8 && sx) return fail(ARIA_ERR_INVALID_ARG, "sx is for W8A8 only");
+  for (const void* q : {X, static_cast<const void*>(sx), Wq, scales, bias,
+                        static_cast<const void*>(steer_vec), static_cast<const void*>(Y)})
+    if (q && !aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  return qgemm_impl(kind, M, N, K, X, sx, Wq, scales, bias, steer_vec, alpha, Y,
+                    static_cast<cudaStream_t>(stream));
+}
+
+ARIA_API aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t* Xq,
+                                    const int8_t* Wq, int32_t* C, void* stream) {
+  if (!Xq || !Wq || !C) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(C))
+    return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  return qgemm_impl(aria::kS32, M, N, K, Xq, nullptr, Wq, Wq, nullptr, nullptr, 0.0f, C,
+                    static_cast<cudaStream_t>(stream));
+}
+
+ARIA_API aria_status aria_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned v = 0, site = 0, zero = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, aria::g_status, sizeof(v))) != cudaSuccess)
+    return cuda_fail(e, "read status word");
+  if (v) {
+    cudaMemcpyFromSymbol(&site, aria::g_wait_site, sizeof(site));
+    cudaMemcpyToSymbol(aria::g_status, &zero, sizeof(zero));
+    return fail(ARIA_ERR_TIMEOUT, "a bounded wait ran out in a kernel (site %u)", site);
+  }
+  return ARIA_OK;
+}

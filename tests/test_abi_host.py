@@ -1,0 +1,89 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+- libaria_q.so loads and exports every function declared in include/aria_q.h;
+- argument validation rejects bad calls before touching CUDA.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import int8_int4_b200 as aq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "aria_q.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(aria_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from int8_int4_b200 import build
+    build.build()
+    return aq.load_library()
+
+
+def test_header_declares_the_api():
+    assert set(_declared()) == set(aq.API)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", aq.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert getattr(lib, name)
+    # nothing else leaks out with default visibility
+    assert {e for e in exported if e.startswith("aria_")} == set(_declared())
+
+
+def test_status_strings(lib):
+    for code, name in aq.STATUS.items():
+        assert lib.aria_status_string(code).decode() == name
+
+
+def test_qpack_size(lib):
+    assert aq.qpack_size("q8", 3072, 1024) == (3072 * 1024, 3072 * 4)
+    assert aq.qpack_size("w8a8", 1536, 6144) == (1536 * 6144, 1536 * 4)
+    assert aq.qpack_size("q4", 6144, 1536) == (6144 * 768, 6144 * 48 * 2)
+    with pytest.raises(aq.AriaError) as e:
+        aq.qpack_size("q4", 16, 48)
+    assert e.value.status == 2
+    with pytest.raises(aq.AriaError) as e:
+        aq.qpack_size("q4", 16, 64, group=64)
+    assert e.value.status == 2
+    with pytest.raises(aq.AriaError) as e:
+        aq.qpack_size("q8", 0, 64)
+    assert e.value.status == 1
+
+
+def test_validation_before_launch(lib):
+    P = ctypes.c_void_p
+    # NULL pointers
+    assert lib.aria_qgemm(1, 0, 4, 16, 16, None, None, None, None, None, None, 0.0, None, None) == 1
+    assert lib.aria_act_quant(None, 4, 16, None, None, None) == 1
+    assert lib.aria_qpack(1, 0, None, 16, 16, None, None, None) == 1
+    # misaligned (fake, never dereferenced: the check runs first)
+    bad = P(0x1001)
+    ok = P(0x10000)
+    assert lib.aria_qgemm(1, 0, 4, 16, 16, bad, None, ok, ok, None, None, 0.0, ok, None) == 3
+    assert lib.aria_act_quant(ok, 4, 16, bad, ok, None) == 3
+    # format / argument rules
+    assert lib.aria_qgemm(3, 0, 4, 16, 16, ok, None, ok, ok, None, None, 0.0, ok, None) == 1  # W8A8 w/o sx
+    assert lib.aria_qgemm(1, 0, 4, 16, 16, ok, ok, ok, ok, None, None, 0.0, ok, None) == 1    # sx on q8
+    assert lib.aria_qgemm(2, 16, 4, 16, 256, ok, None, ok, ok, None, None, 0.0, ok, None) == 2  # group
+    assert lib.aria_qgemm(9, 0, 4, 16, 16, ok, None, ok, ok, None, None, 0.0, ok, None) == 1
+    assert b"sx" in lib.aria_last_error_message() or lib.aria_last_error_message()
+
+
+def test_no_cpu_path():
+    import torch
+    with pytest.raises(ValueError):
+        aq.act_quant(torch.zeros(4, 16, dtype=torch.float16))

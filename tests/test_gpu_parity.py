@@ -1,0 +1,270 @@
+"""GPU parity of the CUDA path against the CPU oracle (needs a B200).
+
+Bars (element by element, same seeded inputs on both sides):
+- packed bytes, scales, activation codes and int32 accumulators: bit-exact;
+- W8A8 fp16 outputs: within 1 fp16 ulp (the fp64 epilogue is expected to be
+  bit-exact; the test reports the worst distance);
+- q8 / q4 weight-only fp16 outputs vs the unrounded fp64 reference:
+  max |y - y_ref| <= 1e-2 * max |y_ref| and ||y - y_ref||_F <= 1e-3 * ||y_ref||_F.
+Shapes span several tiles, ragged tails in M, N and K, the degenerate cases
+(M = 1, zero rows, N = K = 16) and, on sampled rows, the full workload sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import int8_int4_b200 as aq
+import oracle
+import synthetic
+
+pytestmark = pytest.mark.gpu
+
+WO_MAXABS = 1e-2
+WO_FROB = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    aq.load_library()   # raises if the CUDA library is missing: no fallback
+    yield
+    aq.device_status()
+
+
+def f16np(t):
+    return t.detach().cpu().numpy()
+
+
+def ulp_dist(a_bits, b_bits):
+    """distance in fp16 ulps between bit patterns (+0 == -0)"""
+    def ordered(b):
+        b = b.astype(np.int32)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+    return np.abs(ordered(a_bits) - ordered(b_bits))
+
+
+def check_wo(y_gpu, y_ref):
+    y = y_gpu.astype(np.float64)
+    err = np.abs(y - y_ref)
+    scale = np.abs(y_ref).max()
+    assert err.max() <= WO_MAXABS * scale, (err.max(), scale)
+    assert np.linalg.norm(y - y_ref) <= WO_FROB * np.linalg.norm(y_ref)
+
+
+def sample_rows(M, k, seed=0):
+    if M <= k:
+        return np.arange(M)
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, M - 1], rng.choice(M, k - 2, replace=False)]))
+
+
+# ------------------------------------------------------------------ packs --
+
+@pytest.mark.parametrize("N,K", [(256, 256), (48, 48), (3072, 1024), (1024, 4096),
+                                 (4608, 1536), (1536, 6144), (130, 2064)])
+def test_pack_q8_bit_exact(N, K):
+    W = synthetic.weight(f"gpu/pq8/{N}x{K}", N, K, outlier_frac=0.001)
+    W[1] = 0                                   # an all-zero channel
+    Wq, s = aq.qpack("q8", W.cuda())
+    rq, rs = oracle.pack_q8(W.numpy())
+    assert np.array_equal(Wq.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K", [(16, 64), (64, 96), (4608, 1536), (1536, 6144), (6144, 1536), (40, 256)])
+def test_pack_q4_bit_exact(N, K):
+    W = synthetic.weight(f"gpu/pq4/{N}x{K}", N, K, outlier_frac=0.001)
+    W[0, :32] = 0                              # an all-zero group
+    P, S = aq.qpack("q4", W.cuda())
+    rp, rs = oracle.pack_q4(W.numpy())
+    assert np.array_equal(P.cpu().numpy(), rp)
+    assert np.array_equal(S.cpu().numpy().view(np.uint16), rs)
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (432, 1536), (432, 6144), (4096, 1536), (4096, 6144),
+                                 (7, 8208), (33, 2064)])
+def test_act_quant_bit_exact(M, K):
+    X = synthetic.activation(f"gpu/aq/{M}x{K}", M, K, outlier_channel_frac=0.01)
+    if M > 2:
+        X[2] = 0
+    Xq, sx = aq.act_quant(X.cuda())
+    rq, rs = oracle.act_quant(X.numpy())
+    assert np.array_equal(Xq.cpu().numpy(), rq)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+# ------------------------------------------------------------ int8 GEMM ---
+
+def _w8a8_inputs(M, N, K, key):
+    W = synthetic.weight(f"{key}/W", N, K)
+    X = synthetic.activation(key, M, K, outlier_channel_frac=0.01)
+    Wq, sw = aq.qpack("q8", W.cuda())
+    Xq, sx = aq.act_quant(X.cuda())
+    return X, W, Xq, sx, Wq, sw
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 16, 16), (1, 128, 128), (64, 256, 256), (300, 400, 1040),
+                                   (432, 1536, 1536), (257, 128, 4096), (2, 4608, 1536)])
+def test_s32_bit_exact(M, N, K):
+    X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, f"gpu/s32/{M}x{N}x{K}")
+    C = aq.qgemm_s32(Xq, Wq)
+    ref = oracle.gemm_s32(Xq.cpu().numpy(), Wq.cpu().numpy())
+    assert np.array_equal(C.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 6144, 1536), (4096, 1536, 6144), (432, 4608, 1536)])
+def test_s32_full_size_sampled(M, N, K):
+    X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, f"gpu/s32f/{M}x{N}x{K}")
+    C = aq.qgemm_s32(Xq, Wq)
+    rows = sample_rows(M, 12)
+    ref = oracle.gemm_s32(Xq.cpu().numpy(), Wq.cpu().numpy(), rows=rows)
+    assert np.array_equal(C.cpu().numpy()[rows], ref)
+
+
+@pytest.mark.parametrize("M,N,K,bias,steer", [
+    (64, 256, 256, True, False), (300, 400, 1040, True, True), (432, 1536, 1536, False, True),
+    (1, 16, 16, True, True), (432, 6144, 1536, False, False)])
+def test_w8a8_within_one_ulp(M, N, K, bias, steer):
+    key = f"gpu/w8a8/{M}x{N}x{K}"
+    X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, key)
+    b = synthetic.bias(key, N) if bias else None
+    v = synthetic.steer_vec(key, N) if steer else None
+    alpha = 0.3 if steer else 0.0
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx, bias=None if b is None else b.cuda(),
+                 steer_vec=None if v is None else v.cuda(), alpha=alpha)
+    ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(),
+                      None if b is None else b.numpy(), None if v is None else v.numpy(), alpha)
+    d = ulp_dist(Y.cpu().numpy().view(np.uint16), ref)
+    assert d.max() <= 1, d.max()
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 6144, 1536), (4096, 1536, 6144), (4096, 4608, 1536)])
+def test_w8a8_full_size_sampled(M, N, K):
+    key = f"gpu/w8a8f/{M}x{N}x{K}"
+    X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, key)
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx)
+    rows = sample_rows(M, 8)
+    ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(), rows=rows)
+    d = ulp_dist(Y.cpu().numpy().view(np.uint16)[rows], ref)
+    assert d.max() <= 1, d.max()
+
+
+# ------------------------------------------------------- weight-only GEMM ---
+
+def _wo(fmt, M, N, K, key, bias=False, steer=False, rows=None, outliers=0.0):
+    W = synthetic.weight(f"{key}/W", N, K, outlier_frac=outliers)
+    X = synthetic.activation(key, M, K)
+    b = synthetic.bias(key, N) if bias else None
+    v = synthetic.steer_vec(key, N) if steer else None
+    alpha = 0.3 if steer else 0.0
+    Wq, sc = aq.qpack(fmt, W.cuda())
+    Y = aq.qgemm(fmt, X.cuda(), Wq, sc, bias=None if b is None else b.cuda(),
+                 steer_vec=None if v is None else v.cuda(), alpha=alpha)
+    scn = sc.cpu().numpy()
+    ref = oracle.wo_ref(fmt, X.numpy(), Wq.cpu().numpy(), scn if fmt == "q8" else scn.view(np.uint16),
+                        None if b is None else b.numpy(), None if v is None else v.numpy(), alpha,
+                        rows=rows)
+    y = f16np(Y)
+    return (y if rows is None else y[rows]), ref
+
+
+def test_tiny_q8_config():
+    """W [256,256] ~N(0,0.02^2), X [64,256] ~N(0,1), bias ~N(0,0.01^2), seed 0."""
+    d = synthetic.tiny_q8()
+    Wq, s = aq.qpack("q8", d["W"].cuda())
+    rq, rs = oracle.pack_q8(d["W"].numpy())
+    assert np.array_equal(Wq.cpu().numpy(), rq) and np.array_equal(s.cpu().numpy(), rs)
+    Y = aq.qgemm("q8", d["X"].cuda(), Wq, s, bias=d["bias"].cuda())
+    check_wo(f16np(Y), oracle.wo_ref("q8", d["X"].numpy(), rq, rs, d["bias"].numpy()))
+
+
+@pytest.mark.parametrize("M,N,K,bias,steer", [
+    (16, 16, 16, False, False), (1, 128, 128, True, False), (64, 256, 256, True, True),
+    (300, 400, 1040, True, True), (17, 3072, 1024, False, False), (432, 1024, 1024, True, False),
+    (5, 1024, 4096, False, True)])
+def test_q8_weight_only(M, N, K, bias, steer):
+    y, ref = _wo("q8", M, N, K, f"gpu/q8/{M}x{N}x{K}", bias, steer)
+    check_wo(y, ref)
+
+
+@pytest.mark.parametrize("name", ["qkv", "out", "up", "down"])
+@pytest.mark.parametrize("M", [1, 16, 432])
+def test_q8_d1024_block(name, M):
+    W, X = synthetic.q8_block_d1024(name, M)
+    Wq, s = aq.qpack("q8", W.cuda())
+    Y = aq.qgemm("q8", X.cuda(), Wq, s)
+    rows = sample_rows(M, 24)
+    ref = oracle.wo_ref("q8", X.numpy(), Wq.cpu().numpy(), s.cpu().numpy(), rows=rows)
+    check_wo(f16np(Y)[rows], ref)
+
+
+@pytest.mark.parametrize("M,N,K,bias,steer", [
+    (16, 16, 256, False, False), (1, 128, 256, True, False), (64, 256, 512, True, True),
+    (300, 400, 1024, True, True), (8, 1536, 6144, False, False)])
+def test_q4_weight_only(M, N, K, bias, steer):
+    y, ref = _wo("q4", M, N, K, f"gpu/q4/{M}x{N}x{K}", bias, steer, outliers=0.001)
+    check_wo(y, ref)
+
+
+@pytest.mark.parametrize("name", ["qkv", "out", "up", "down"])
+@pytest.mark.parametrize("M", [1, 8, 432])
+def test_q4_d1536_block(name, M):
+    W, X = synthetic.q4_d1536(name, M)
+    P, S = aq.qpack("q4", W.cuda())
+    Y = aq.qgemm("q4", X.cuda(), P, S)
+    rows = sample_rows(M, 16)
+    ref = oracle.wo_ref("q4", X.numpy(), P.cpu().numpy(), S.cpu().numpy().view(np.uint16), rows=rows)
+    check_wo(f16np(Y)[rows], ref)
+
+
+# ---------------------------------------------------------- epilogue rules --
+
+@pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
+def test_alpha_zero_is_bit_identical(fmt):
+    M, N, K = 96, 512, 1024
+    W = synthetic.weight(f"gpu/a0/{fmt}/W", N, K)
+    X = synthetic.activation(f"gpu/a0/{fmt}", M, K).cuda()
+    v = synthetic.steer_vec(f"gpu/a0/{fmt}", N).cuda()
+    b = synthetic.bias(f"gpu/a0/{fmt}", N).cuda()
+    Wq, sc = aq.qpack("q8" if fmt == "w8a8" else fmt, W.cuda())
+    kw = {}
+    if fmt == "w8a8":
+        X, sx = aq.act_quant(X)
+        kw["sx"] = sx
+    base = aq.qgemm(fmt, X, Wq, sc, bias=b, **kw)
+    assert torch.equal(aq.qgemm(fmt, X, Wq, sc, bias=b, steer_vec=v, alpha=0.0, **kw).view(torch.int16),
+                       base.view(torch.int16))
+    assert torch.equal(aq.qgemm(fmt, X, Wq, sc, bias=b, steer_vec=None, alpha=0.5, **kw).view(torch.int16),
+                       base.view(torch.int16))
+    steered = aq.qgemm(fmt, X, Wq, sc, bias=b, steer_vec=v, alpha=0.3, **kw)
+    diff = (steered.double() - base.double()) - 0.3 * v.double()[None, :]
+    assert diff.abs().max().item() < 2e-3          # y + alpha*v, up to fp16 rounding
+
+
+@pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
+def test_deterministic_split_k(fmt):
+    M, N, K = 1, 1024, 4096                        # few tiles: split-K across a cluster
+    W = synthetic.weight(f"gpu/det/{fmt}/W", N, K)
+    X = synthetic.activation(f"gpu/det/{fmt}", M, K).cuda()
+    Wq, sc = aq.qpack("q8" if fmt == "w8a8" else fmt, W.cuda())
+    kw = {}
+    if fmt == "w8a8":
+        X, sx = aq.act_quant(X)
+        kw["sx"] = sx
+    ys = [aq.qgemm(fmt, X, Wq, sc, **kw).view(torch.int16) for _ in range(3)]
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
+
+
+def test_zero_inputs_give_bias():
+    M, N, K = 8, 256, 512
+    b = synthetic.bias("gpu/zero", N).cuda()
+    W = synthetic.weight("gpu/zero/W", N, K).cuda()
+    X = torch.zeros(M, K, dtype=torch.float16, device="cuda")
+    for fmt in ("q8", "q4"):
+        Wq, sc = aq.qpack(fmt, W)
+        Y = aq.qgemm(fmt, X, Wq, sc, bias=b)
+        assert torch.equal(Y.float(), b.float().expand(M, N))
+    Wq, sw = aq.qpack("q8", W)
+    Xq, sx = aq.act_quant(X)
+    assert not Xq.any() and not sx.any()
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx, bias=b)
+    assert torch.equal(Y.float(), b.float().expand(M, N))
