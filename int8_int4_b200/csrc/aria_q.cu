@@ -100,6 +100,7 @@ DevInfo dev_info() {
 struct Plan {
   aria::GemmParams p;
   dim3 grid;
+  int threads;
   size_t smem;
 };
 
@@ -120,18 +121,25 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.BN = bn;
   const int nt = static_cast<int>((N + kTileN - 1) / kTileN);
   const int64_t tiles = static_cast<int64_t>(nt) * mt;
-  if (mt > 65535 || nt > 65535) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
+  if (tiles > (int64_t{1} << 30)) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
+  p.tiles_n = nt;
+  p.tiles = static_cast<int>(tiles);
 
+  // split-K upper bound; the launcher lowers it until the clusters fit in one wave
   int splits = 1;
   if (tiles < di.sms) splits = static_cast<int>(std::min<int64_t>(8, di.sms / tiles));
   splits = std::max(1, std::min(splits, p.units));
   p.splits = splits;
 
-  p.x_stage = static_cast<uint32_t>(bn) * 128u;
   const bool dq = (kind == kQ8 || kind == kQ4);
+  const uint32_t out_bytes = kind == kS32 ? 4 : 2;
+  const uint32_t epi_warps = dq ? 4 : 8;
+  const uint32_t stage_bytes = epi_warps * 2 * kEpiRows * 32 * out_bytes;  // 2 store boxes per warp
+  const uint32_t sxd_bytes = 256 * 4;
+  p.x_stage = static_cast<uint32_t>(bn) * 128u;
   p.raw_stage = kind == kQ8 ? kATile : (kind == kQ4 ? kATile + kQ4ScaleTile : 0);
   p.raw_stage = (p.raw_stage + 1023u) & ~1023u;
-  const int64_t budget = static_cast<int64_t>(di.smem_optin) - 1024 - 1024;  // align + barriers
+  const int64_t budget = static_cast<int64_t>(di.smem_optin) - 1024 - 512 - stage_bytes - sxd_bytes;
   int nr = 0, na = 0, nx = 0;
   if (dq) {
     na = bn > 128 ? 3 : 4;
@@ -152,55 +160,100 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.off_raw = 0;
   p.off_a = p.off_raw + nr * p.raw_stage;
   p.off_x = p.off_a + na * kATile;
-  p.off_bar = p.off_x + nx * p.x_stage;
-  if (splits > 1 && static_cast<uint32_t>(bn) * 512u > p.off_bar)
-    return fail(ARIA_ERR_UNSUPPORTED, "split-K buffer does not fit");
-  const uint32_t nbar = 2 * (nr + na + nx) + 1;
+  p.off_stage = p.off_x + nx * p.x_stage;
+  p.off_sxd = p.off_stage + stage_bytes;
+  p.off_bar = p.off_sxd + sxd_bytes;
+  if (static_cast<uint32_t>(bn) * 512u > p.off_stage) p.splits = splits = 1;  // no room to reduce
+  const uint32_t nbar = 2 * (nr + na + nx) + 5;
   const size_t smem = 1024 + p.off_bar + nbar * 8 + 16;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(bn)) cols <<= 1;
-  p.tmem_cols = cols;
+  if (smem > static_cast<size_t>(di.smem_optin)) return fail(ARIA_ERR_UNSUPPORTED, "shared memory plan too large");
 
   out->p = p;
-  out->grid = dim3(splits, nt, mt);
+  out->grid = dim3(static_cast<unsigned>(std::min<int64_t>(tiles, di.sms)), 1, 1);
+  out->threads = 384;
   out->smem = smem;
   return ARIA_OK;
 }
 
+// programmatic dependent launch: the kernel may start while the previous
+// kernel in the stream drains; it waits (griddepcontrol.wait) before touching
+// global memory
+void set_pdl(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr) {
+  attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs++;
+  cfg.attrs = attr;
+}
+
+// how many clusters of `size` CTAs of this kernel can be resident at once
+// (cached per size and shared-memory footprint; queried outside any capture
+// on first use)
+template <int KIND>
+int max_clusters(int size, int threads, size_t smem) {
+  static std::mutex mu;
+  static int cache_size[64], cache_n[64];
+  static size_t cache_smem[64];
+  static int used = 0;
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache_size[i] == size && cache_smem[i] == smem) return cache_n[i];
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(size, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = size;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, aria::qgemm_kernel<KIND>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (used < 64) {
+    cache_size[used] = size;
+    cache_smem[used] = smem;
+    cache_n[used] = n;
+    ++used;
+  }
+  return n;
+}
+
 template <int KIND>
 aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap& ts,
-                        const CUtensorMap& tx, cudaStream_t st) {
+                        const CUtensorMap& tx, const CUtensorMap& ty, cudaStream_t st) {
   auto kfn = aria::qgemm_kernel<KIND>;
-  static int configured_for = -1;
-  static std::mutex mu;
-  {
-    std::lock_guard<std::mutex> g(mu);
-    int dev = 0;
-    cudaGetDevice(&dev);
-    // set once per process and device-independent: the attribute is per function
-    if (configured_for != dev) {
-      cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           dev_info().smem_optin);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-      configured_for = dev;
-    }
-  }
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    dev_info().smem_optin);
+  });
+  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute");
+  aria::GemmParams prm = pl.p;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
-  cfg.blockDim = dim3(aria::kGemmThreads, 1, 1);
+  cfg.blockDim = dim3(pl.threads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.numAttrs = 0;
-  if (pl.p.splits > 1) {
+  // largest split whose clusters are all co-resident (one wave)
+  while (prm.splits > 1 && max_clusters<KIND>(prm.splits, pl.threads, pl.smem) < prm.tiles) --prm.splits;
+  if (prm.splits > 1) {
+    cfg.gridDim = dim3(prm.splits, prm.tiles, 1);
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.p.splits;
+    attr[0].val.clusterDim.x = prm.splits;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.attrs = attr;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, pl.p);
+  set_pdl(cfg, attr);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, ty, prm);
   if (e != cudaSuccess) return cuda_fail(e, "qgemm launch");
   return ARIA_OK;
 }
@@ -262,18 +315,25 @@ ARIA_API aria_status aria_qpack(aria_format fmt, int group, const void* W, int64
   if (!aligned16(W) || !aligned16(Wq) || !aligned16(scales))
     return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  cfg.stream = st;
+  set_pdl(cfg, attr);
+  cudaError_t e;
   if (fmt == ARIA_FMT_Q4) {
     const int64_t nchunk = N * (K / 8);
-    const int64_t blocks = std::min<int64_t>((nchunk + 255) / 256, 148 * 16);
-    aria::pack_q4_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        static_cast<const __half*>(W), nchunk, static_cast<uint32_t*>(Wq), static_cast<__half*>(scales));
+    const int64_t blocks = std::min<int64_t>((nchunk + 255) / 256, int64_t{dev_info().sms} * 16);
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(256);
+    e = cudaLaunchKernelEx(&cfg, aria::pack_q4_kernel, static_cast<const __half*>(W), nchunk,
+                           static_cast<uint32_t*>(Wq), static_cast<__half*>(scales));
   } else {
     if (K % 16) return fail(ARIA_ERR_UNSUPPORTED, "q8 needs K % 16 == 0");
-    aria::row_quant_i8_kernel<<<static_cast<unsigned>(N), aria::kRowThreads, 0, st>>>(
-        static_cast<const __half*>(W), static_cast<int>(K), static_cast<int8_t*>(Wq),
-        static_cast<float*>(scales));
+    cfg.gridDim = dim3(static_cast<unsigned>(N));
+    cfg.blockDim = dim3(aria::kRowThreads);
+    e = cudaLaunchKernelEx(&cfg, aria::row_quant_i8_kernel, static_cast<const __half*>(W),
+                           static_cast<int>(K), static_cast<int8_t*>(Wq), static_cast<float*>(scales));
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   return ARIA_OK;
 }
@@ -286,10 +346,14 @@ ARIA_API aria_status aria_act_quant(const void* X, int64_t M, int64_t K, int8_t*
   if (K % 16) return fail(ARIA_ERR_UNSUPPORTED, "K must be a multiple of 16");
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(sx))
     return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
-  aria::row_quant_i8_kernel<<<static_cast<unsigned>(M), aria::kRowThreads, 0,
-                              static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __half*>(X), static_cast<int>(K), Xq, sx);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cfg.gridDim = dim3(static_cast<unsigned>(M));
+  cfg.blockDim = dim3(aria::kRowThreads);
+  set_pdl(cfg, attr);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, aria::row_quant_i8_kernel, static_cast<const __half*>(X),
+                                     static_cast<int>(K), Xq, sx);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return ARIA_OK;
 }
@@ -323,6 +387,17 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
     if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, bn,
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   }
+  CUtensorMap ty;
+  std::memset(&ty, 0, sizeof(ty));
+  if (pl.p.splits == 1) {
+    if (kind == kS32) {
+      if ((s = make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, M, N, 32, kEpiRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
+    } else {
+      if ((s = make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, kEpiRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
+    }
+  }
   pl.p.sw = static_cast<const float*>(kind == kQ4 ? nullptr : scales);
   pl.p.sx = sx;
   pl.p.bias = static_cast<const __half*>(bias);
@@ -331,10 +406,10 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
   pl.p.Y = Y;
   if (!pl.p.steer) pl.p.alpha = 0.0f;
   switch (kind) {
-    case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, st);
-    case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, st);
-    case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, st);
-    case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, st);
+    case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, ty, st);
+    case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, ty, st);
+    case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, ty, st);
+    case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, ty, st);
   }
   return fail(ARIA_ERR_INVALID_ARG, "unknown kind");
 }

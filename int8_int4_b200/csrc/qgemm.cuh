@@ -10,19 +10,22 @@
 // without padding the token dimension to 128. Both operands are K-major in
 // the 128-byte swizzled shared-memory layout.
 //
-// Warp roles (256 threads, one CTA per SM):
-//   warp 0      TMA producer of weight tiles (raw packed bytes for q8/q4, the
-//               int8 A operand itself for W8A8)
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warp 2      TMA producer of activation tiles (fp16 for q8/q4, int8 W8A8)
-//   warps 4..7  q8/q4: dequantise raw weights into fp16 A tiles (one weight
-//               row per thread, exact int8->fp16, fp16 code*scale for q4);
-//               then the epilogue: TMEM -> registers -> scale, bias, steer ->
-//               fp16 stores (fp64 arithmetic for W8A8).
-// Split-K: when the output tiles are too few to cover the SMs, a cluster of S
-// CTAs shares one output tile, each taking a contiguous K range; partial
-// accumulators are summed through distributed shared memory in fixed rank
-// order (deterministic, no global scratch).
+// Persistent, warp-specialised CTA (one per SM):
+//   warp 0       TMA producer of weight tiles (raw packed bytes for q8/q4, the
+//                int8 A operand itself for W8A8)
+//   warp 1       TMEM allocator (two accumulator buffers) and the single-thread
+//                tcgen05.mma issuer
+//   warp 2       TMA producer of activation tiles
+//   warps 4..7   epilogue: TMEM -> registers -> scale, bias, steer -> fp16 ->
+//                shared staging -> TMA bulk store; overlaps the next tile's
+//                mainloop through the second accumulator buffer
+//   warps 8..11  q8/q4 only: dequantise raw weights into fp16 A tiles (one
+//                weight row per thread; exact int8 -> fp16; fp16 code*scale for q4)
+// Rings of shared-memory stages with mbarriers connect the roles; every wait
+// is bounded. Split-K (few output tiles): a cluster of S CTAs shares one tile,
+// each taking a contiguous K range, and partial accumulators are summed
+// through distributed shared memory in fixed rank order (deterministic, no
+// global scratch).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -34,26 +37,27 @@ namespace aria {
 
 enum GemmKind : int { kQ8 = 1, kQ4 = 2, kW8A8 = 3, kS32 = 4 };
 
-constexpr int kGemmThreads = 256;
-constexpr int kTileN = 128;            // weight rows per tile (MMA M)
-constexpr uint32_t kATile = 16384;     // 128 rows x 128 bytes
+constexpr int kTileN = 128;              // weight rows per tile (MMA M)
+constexpr uint32_t kATile = 16384;       // 128 rows x 128 bytes
 constexpr uint32_t kQ4ScaleTile = 2048;  // 128 rows x 8 fp16 scales
+constexpr uint32_t kAccCols = 256;       // TMEM columns per accumulator buffer
+constexpr int kEpiRows = 16;             // tokens per epilogue store box
 
 struct GemmParams {
   int M, N, K;
   int BN;                 // tokens per tile (MMA N): multiple of 16, <= 256
   int units;              // K units: 128 (q8, W8A8) or 256 (q4) elements
-  int splits;             // CTAs per cluster along K
+  int splits;             // CTAs per cluster along K (1 = persistent over tiles)
+  int tiles_n, tiles;     // weight-row tiles, total output tiles
   int n_raw, n_a, n_x;    // ring depths
-  uint32_t off_raw, off_a, off_x, off_bar;
+  uint32_t off_raw, off_a, off_x, off_stage, off_sxd, off_bar;
   uint32_t raw_stage, x_stage;
-  uint32_t tmem_cols;
   const float* sw;        // per-channel weight scale (q8, W8A8)
   const float* sx;        // per-token activation scale (W8A8)
   const __half* bias;     // [N] or null
   const float* steer;     // [N] or null (null also when alpha == 0)
   float alpha;
-  void* Y;                // fp16 [M,N], or int32 [M,N] for kS32
+  void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
 template <int KIND>
@@ -62,6 +66,10 @@ struct KindTraits {
   static constexpr bool kF16 = kDequant;                    // MMA kind::f16 vs kind::i8
   static constexpr int kKbPerUnit = KIND == kQ8 ? 2 : (KIND == kQ4 ? 4 : 1);
   static constexpr int kXElemsPerKb = kF16 ? 64 : 128;      // 128 bytes of K per row
+  static constexpr int kThreads = 384;
+  static constexpr int kEpiWarps = kDequant ? 4 : 8;   // W8A8 / S32 use warps 8..11 for the epilogue too
+  static constexpr uint32_t kOutBytes = KIND == kS32 ? 4 : 2;
+  static constexpr uint32_t kStageBuf = kEpiRows * 32 * kOutBytes;  // one warp's store box
 };
 
 // ---------------------------------------------------------------- dequant ---
@@ -105,25 +113,121 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t j) {
 }
 
 // ---------------------------------------------------------------- epilogue --
+// Per output channel n (one per epilogue thread), the constants of the fused
+// epilogue, loaded once per tile.
 template <int KIND>
-__device__ __forceinline__ __half epi_value(uint32_t acc_bits, int m, int n, const GemmParams& p) {
+struct RowConst {
+  float sw = 0.0f, bias = 0.0f, alpha = 0.0f, v = 0.0f;  // all formats (W8A8: fp32 copies)
+  float av_hi = 0.0f, av_lo = 0.0f;                      // W8A8: alpha*v = av_hi + av_lo exactly
+  bool has_bias = false, has_steer = false;
+};
+
+template <int KIND>
+__device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) {
+  RowConst<KIND> c;
+  if (n >= p.N) return c;
+  c.has_bias = p.bias != nullptr;
+  c.has_steer = p.steer != nullptr;
   if constexpr (KIND == kW8A8) {
-    // fp64: ((acc * s_x) * s_w) + bias + alpha*v, each step rounded once, no
-    // contraction, then one rounding to fp16
-    double t = __dmul_rn(__dmul_rn(static_cast<double>(static_cast<int32_t>(acc_bits)),
-                                   static_cast<double>(__ldg(p.sx + m))),
-                         static_cast<double>(__ldg(p.sw + n)));
-    if (p.bias) t = __dadd_rn(t, static_cast<double>(__half2float(p.bias[n])));
-    if (p.steer)
-      t = __dadd_rn(t, __dmul_rn(static_cast<double>(p.alpha), static_cast<double>(__ldg(p.steer + n))));
-    return __double2half(t);
+    c.sw = __ldg(p.sw + n);
+    if (c.has_bias) c.bias = __half2float(p.bias[n]);
+    if (c.has_steer) {
+      c.alpha = p.alpha;
+      c.v = __ldg(p.steer + n);
+      c.av_hi = __fmul_rn(c.alpha, c.v);
+      c.av_lo = __fmaf_rn(c.alpha, c.v, -c.av_hi);  // exact remainder of the product
+    }
   } else {
-    float y = __uint_as_float(acc_bits);
-    if constexpr (KIND == kQ8) y = __fmul_rn(y, __ldg(p.sw + n));
-    if (p.bias) y = __fadd_rn(y, __half2float(p.bias[n]));
-    if (p.steer) y = __fmaf_rn(p.alpha, __ldg(p.steer + n), y);
-    return __float2half_rn(y);
+    if constexpr (KIND == kQ8) c.sw = __ldg(p.sw + n);
+    if (c.has_bias) c.bias = __half2float(p.bias[n]);
+    if (c.has_steer) {
+      c.alpha = p.alpha;
+      c.v = __ldg(p.steer + n);
+    }
   }
+  return c;
+}
+
+// W8A8 reference sequence: ((acc * s_x) * s_w) + bias + alpha*v in fp64, each
+// step rounded once (no contraction), then one rounding to fp16.
+__device__ __noinline__ __half epi_w8a8_fp64(int32_t acc, float sx, const RowConst<kW8A8>& c) {
+  double t = __dmul_rn(__dmul_rn(static_cast<double>(acc), static_cast<double>(sx)),
+                       static_cast<double>(c.sw));
+  if (c.has_bias) t = __dadd_rn(t, static_cast<double>(c.bias));
+  if (c.has_steer)  // a product of two fp32 values is exact in fp64
+    t = __dadd_rn(t, __dmul_rn(static_cast<double>(c.alpha), static_cast<double>(c.v)));
+  return __double2half(t);
+}
+
+// Knuth's two-sum: s + e == a + b exactly
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+  s = __fadd_rn(a, b);
+  const float bb = __fsub_rn(s, a);
+  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+
+// The same value, rounded to fp16, without fp64 arithmetic. The exact real
+// value E = acc*s_x*s_w + bias + alpha*v is carried as an unevaluated sum
+// yh + yl of two fp32 numbers (error-free products by fma, error-free sums by
+// two-sum), accurate to about 2^-46 relative. Rounding E to fp16 then needs
+// only yh, except when yh lies exactly on a midpoint between two fp16
+// values, where the sign of yl decides. The result equals the fp64
+// reference except if E lies within ~2^-46 of an fp16 midpoint (both are
+// then within one fp16 ulp). |acc| >= 2^22 takes the fp64 sequence.
+__device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst<kW8A8>& c) {
+  if (acc <= -(1 << 22) || acc >= (1 << 22)) return epi_w8a8_fp64(acc, sx, c);
+  const float a = __fsub_rn(__int_as_float(acc + 0x4B400000), 12582912.0f);  // exact int -> float
+  const float ph = __fmul_rn(sx, c.sw);
+  const float pl = __fmaf_rn(sx, c.sw, -ph);        // sx*sw == ph + pl
+  float yh = __fmul_rn(a, ph);
+  float yl = __fmaf_rn(a, ph, -yh);                 // a*ph == yh + yl
+  yl = __fmaf_rn(a, pl, yl);                        // + a*pl (error ~2^-48 |yh|)
+  float e;
+  if (c.has_bias) {
+    two_sum(yh, c.bias, yh, e);
+    yl = __fadd_rn(yl, e);
+  }
+  if (c.has_steer) {
+    two_sum(yh, c.av_hi, yh, e);
+    yl = __fadd_rn(yl, __fadd_rn(e, c.av_lo));
+  }
+  const float s = __fadd_rn(yh, yl);                // renormalise: |yl| <= ulp(yh)/2
+  yl = __fsub_rn(yl, __fsub_rn(s, yh));
+  yh = s;
+  __half h = __float2half_rn(yh);
+  // midpoint case: |yh| exactly halfway between |h| and its neighbour
+  const float ay = fabsf(yh);
+  const float ar = fabsf(__half2float(h));
+  const float d = __fsub_rn(ay, ar);                // exact (Sterbenz, or ar == 0)
+  if (d != 0.0f && yl != 0.0f && ar < 65504.0f) {
+    const uint32_t hb = __half_as_ushort(h) & 0x7FFFu;
+    float half_gap;
+    if (hb < 0x0400u) {
+      half_gap = 0x1p-25f;                          // zero / subnormal spacing 2^-24
+    } else {
+      const int e16 = static_cast<int>(hb >> 10) - 15;
+      const bool down_binade = (d < 0.0f) && ((hb & 0x3FFu) == 0u) && hb > 0x0400u;
+      half_gap = ldexpf(1.0f, e16 - (down_binade ? 12 : 11));
+    }
+    if (fabsf(d) == half_gap) {
+      const float yl_mag = yh < 0.0f ? -yl : yl;    // yl measured away from zero
+      if ((yl_mag > 0.0f) == (d > 0.0f)) {
+        const uint32_t nb = d > 0.0f ? hb + 1u : hb - 1u;
+        h = __ushort_as_half(static_cast<unsigned short>((__half_as_ushort(h) & 0x8000u) | nb));
+      }
+    }
+  }
+  return h;
+}
+
+// q8 / q4: fp32, (acc * s_w) + bias, then + alpha*v[n] (one fma), one rounding to fp16
+template <int KIND>
+__device__ __forceinline__ __half epi_wo(float acc, const RowConst<KIND>& c) {
+  float y = acc;
+  if constexpr (KIND == kQ8) y = __fmul_rn(y, c.sw);
+  if (c.has_bias) y = __fadd_rn(y, c.bias);
+  if (c.has_steer) y = __fmaf_rn(c.alpha, c.v, y);
+  return __float2half_rn(y);
 }
 
 template <int KIND>
@@ -136,9 +240,10 @@ __device__ __forceinline__ uint32_t reduce_add(uint32_t a, uint32_t b) {
 
 // ------------------------------------------------------------------ kernel --
 template <int KIND>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
-                 const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                 const GemmParams p) {
   using T = KindTraits<KIND>;
   extern __shared__ uint8_t dyn_smem[];
   // 1024-byte alignment of the shared-window address (128-byte swizzle atoms)
@@ -147,9 +252,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rank = p.splits > 1 ? static_cast<int>(cluster_ctarank()) : 0;
-  const int n0 = blockIdx.y * kTileN;
-  const int m0 = blockIdx.z * p.BN;
+  const bool split = p.splits > 1;
+  const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
+  const int tile0 = split ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+  const int tstep = split ? static_cast<int>(gridDim.y) : static_cast<int>(gridDim.x);
   const int u_begin = static_cast<int>(static_cast<int64_t>(p.units) * rank / p.splits);
   const int u_end = static_cast<int>(static_cast<int64_t>(p.units) * (rank + 1) / p.splits);
   const int nu = u_end - u_begin;
@@ -158,6 +264,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* raw = smem + p.off_raw;
   uint8_t* abuf = smem + p.off_a;
   uint8_t* xbuf = smem + p.off_x;
+  uint8_t* stage = smem + p.off_stage;
+  float* sxs = reinterpret_cast<float*>(smem + p.off_sxd);   // s_x of the current m-tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + p.n_raw;
@@ -165,8 +273,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* a_empty = a_full + p.n_a;
   uint64_t* x_full = a_empty + p.n_a;
   uint64_t* x_empty = x_full + p.n_x;
-  uint64_t* acc_full = x_empty + p.n_x;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = x_empty + p.n_x;   // [2]
+  uint64_t* acc_empty = acc_full + 2;     // [2]
+  uint64_t* mma_drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -182,7 +292,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(x_full + i, 1);
       mbar_init(x_empty + i, 1);
     }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, T::kEpiWarps);
+    }
+    mbar_init(mma_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -190,48 +304,66 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
     if constexpr (KIND == kQ4) prefetch_tmap(&tmS);
+    if (!split) prefetch_tmap(&tmY);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Weights start moving into L2 while the preceding kernel drains: an L2
+  // prefetch is safe even if that kernel were still writing them (L2 is
+  // coherent), and the shared-memory loads below only start after the wait.
+  if (warp == 0 && lane == 0 && tile0 < p.tiles) {
+    const int n0 = (tile0 % p.tiles_n) * kTileN;
+    const int npf = nu < 4 ? nu : 4;
+    for (int i = 0; i < npf; ++i) {
+      tma_prefetch_2d(&tmW, (u_begin + i) * 128, n0);
+      if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
+    }
+  }
+  // Inputs may come from the preceding kernel in the stream (programmatic
+  // dependent launch): everything above overlapped its tail; nothing below
+  // reads or writes global memory before it has completed.
+  pdl_wait();
+  pdl_launch_dependents();
 
-  // counters kept for the teardown drain of copies in flight
-  int issued_w = 0, issued_x = 0;
+  int issued_w = 0, issued_x = 0;  // kept for the teardown drain
 
   if (warp == 0) {
     // ------------------------------------------------ weight tile producer
     if (lane == 0) {
-      const uint64_t pol = policy_evict_first();  // weights are read once
-      if constexpr (T::kDequant) {
-        for (int i = 0; i < nu; ++i) {
-          const int s = i % p.n_raw;
-          const uint32_t ph = (i / p.n_raw) & 1;
-          if (!mbar_wait(raw_empty + s, ph ^ 1, abort_flag, 1)) break;
-          uint8_t* dst = raw + s * p.raw_stage;
-          const int u = u_begin + i;
-          if constexpr (KIND == kQ8) {
-            mbar_arrive_expect_tx(raw_full + s, kATile);
-            tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);
-          } else {
-            mbar_arrive_expect_tx(raw_full + s, kATile + kQ4ScaleTile);
-            tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);       // 256 k as bytes
-            tma_load_2d(&tmS, raw_full + s, dst + kATile, u * 8, n0, pol);  // 8 group scales
+      const uint64_t pol = policy_evict_first();  // weights are read once per m-tile
+      bool ok = true;
+      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+        const int n0 = (tile % p.tiles_n) * kTileN;
+        if constexpr (T::kDequant) {
+          for (int i = 0; i < nu; ++i) {
+            const int s = issued_w % p.n_raw;
+            if (!(ok = mbar_wait(raw_empty + s, ((issued_w / p.n_raw) & 1) ^ 1, abort_flag, 1))) break;
+            uint8_t* dst = raw + s * p.raw_stage;
+            const int u = u_begin + i;
+            if constexpr (KIND == kQ8) {
+              mbar_arrive_expect_tx(raw_full + s, kATile);
+              tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);
+            } else {
+              mbar_arrive_expect_tx(raw_full + s, kATile + kQ4ScaleTile);
+              tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);        // 256 k as bytes
+              tma_load_2d(&tmS, raw_full + s, dst + kATile, u * 8, n0, pol);  // 8 group scales
+            }
+            ++issued_w;
           }
-          ++issued_w;
-        }
-      } else {
-        for (int kb = 0; kb < nkb; ++kb) {
-          const int s = kb % p.n_a;
-          const uint32_t ph = (kb / p.n_a) & 1;
-          if (!mbar_wait(a_empty + s, ph ^ 1, abort_flag, 2)) break;
-          mbar_arrive_expect_tx(a_full + s, kATile);
-          tma_load_2d(&tmW, a_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
-          ++issued_w;
+        } else {
+          for (int kb = 0; kb < nkb; ++kb) {
+            const int s = issued_w % p.n_a;
+            if (!(ok = mbar_wait(a_empty + s, ((issued_w / p.n_a) & 1) ^ 1, abort_flag, 2))) break;
+            mbar_arrive_expect_tx(a_full + s, kATile);
+            tma_load_2d(&tmW, a_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
+            ++issued_w;
+          }
         }
       }
     }
@@ -240,166 +372,249 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();   // re-read by every weight tile
       const int kx0 = u_begin * T::kKbPerUnit;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % p.n_x;
-        const uint32_t ph = (kb / p.n_x) & 1;
-        if (!mbar_wait(x_empty + s, ph ^ 1, abort_flag, 3)) break;
-        mbar_arrive_expect_tx(x_full + s, p.x_stage);
-        tma_load_2d(&tmX, x_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
-        ++issued_x;
+      bool ok = true;
+      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+        const int m0 = (tile / p.tiles_n) * p.BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          const int s = issued_x % p.n_x;
+          if (!(ok = mbar_wait(x_empty + s, ((issued_x / p.n_x) & 1) ^ 1, abort_flag, 3))) break;
+          mbar_arrive_expect_tx(x_full + s, p.x_stage);
+          tma_load_2d(&tmX, x_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
+          ++issued_x;
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = T::kF16 ? idesc_f16_f32(p.BN) : idesc_s8_s32(p.BN);
+      int ka = 0, ti = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int sa = kb % p.n_a, sx = kb % p.n_x;
-        ok = mbar_wait(a_full + sa, (kb / p.n_a) & 1, abort_flag, 4) &&
-             mbar_wait(x_full + sx, (kb / p.n_x) & 1, abort_flag, 5);
-        if (!ok) break;
+      for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
+        const int b = ti & 1;
+        if (!(ok = mbar_wait(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9))) break;
         tc_fence_after();
-        const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
-        const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sx * p.x_stage));
+        const uint32_t dt = tmem_base + b * kAccCols;
+        for (int kb = 0; kb < nkb; ++kb, ++ka) {
+          const int sa = ka % p.n_a, sx = ka % p.n_x;
+          ok = mbar_wait(a_full + sa, (ka / p.n_a) & 1, abort_flag, 4) &&
+               mbar_wait(x_full + sx, (ka / p.n_x) & 1, abort_flag, 5);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
+          const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sx * p.x_stage));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
-          if constexpr (T::kF16)
-            umma_f16(tmem_base, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
-          else
-            umma_i8(tmem_base, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+          for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
+            if constexpr (T::kF16)
+              umma_f16(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+            else
+              umma_i8(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+          }
+          umma_commit(a_empty + sa);
+          umma_commit(x_empty + sx);
         }
-        umma_commit(a_empty + sa);
-        umma_commit(x_empty + sx);
+        umma_commit(acc_full + b);  // also fires when nothing was issued
       }
-      umma_commit(acc_full);  // also fires when nothing was issued
+    }
+  } else if (T::kDequant && warp >= 8) {
+    // ------------------------------------------------------ dequantise
+    if constexpr (T::kDequant) {
+      const int t = threadIdx.x - 256;  // weight row within the tile
+      int ir = 0, ia = 0;
+      bool ok = true;
+      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+        for (int i = 0; i < nu && ok; ++i, ++ir) {
+          const int s = ir % p.n_raw;
+          if (!(ok = mbar_wait(raw_full + s, (ir / p.n_raw) & 1, abort_flag, 6))) break;
+          const uint8_t* src = raw + s * p.raw_stage;
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(src + sw128(t, c));
+          uint4 sc = make_uint4(0, 0, 0, 0);
+          if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
+          mbar_arrive(raw_empty + s);
+#pragma unroll
+          for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
+            const int sa = ia % p.n_a;
+            if (!(ok = mbar_wait(a_empty + sa, ((ia / p.n_a) & 1) ^ 1, abort_flag, 7))) break;
+            uint8_t* dst = abuf + sa * kATile;
+            if constexpr (KIND == kQ8) {
+              // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                const uint4 w = v[4 * h + cc];
+                uint4 o0, o1;
+                i8x4_to_h(w.x, o0.x, o0.y);
+                i8x4_to_h(w.y, o0.z, o0.w);
+                i8x4_to_h(w.z, o1.x, o1.y);
+                i8x4_to_h(w.w, o1.z, o1.w);
+                *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc)) = o0;
+                *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc + 1)) = o1;
+              }
+            } else {
+              // raw chunks 2h, 2h+1 (one 32-k group each) -> fp16 chunks 0..7
+              const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
+#pragma unroll
+              for (int g = 0; g < 2; ++g) {
+                const int c = 2 * h + g;
+                const uint32_t spair = scw[c >> 1];
+                const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
+                const uint4 w = v[c];
+                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 0)) = nib8_to_h(w.x, s2);
+                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 1)) = nib8_to_h(w.y, s2);
+                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 2)) = nib8_to_h(w.z, s2);
+                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 3)) = nib8_to_h(w.w, s2);
+              }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(a_full + sa);
+            ++ia;
+          }
+        }
+      }
     }
   } else if (warp >= 4) {
-    const int t = threadIdx.x - 128;  // weight row within the tile == TMEM lane
-    bool ok = true;
-    if constexpr (T::kDequant) {
-      // ------------------------------------------------------ dequantise
-      int ia = 0;
-      for (int i = 0; i < nu && ok; ++i) {
-        const int s = i % p.n_raw;
-        if (!(ok = mbar_wait(raw_full + s, (i / p.n_raw) & 1, abort_flag, 6))) break;
-        const uint8_t* src = raw + s * p.raw_stage;
-        uint4 v[8];
+    // ----------------------------------------------------------- epilogue
+    // kEpiWarps warps; warp e (0-based) reads TMEM lanes 32*(warp%4).. and
+    // takes every (kEpiWarps/4)-th 16-column chunk starting at e/4.
+    const int e = warp - 4;
+    const int nep = T::kEpiWarps * 32;
+    const int te = threadIdx.x - 128;
+    const int t = (warp & 3) * 32 + lane;  // weight row within the tile == TMEM lane
+    const int cgrp = e >> 2, cstep = T::kEpiWarps >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    if (!split) {
+      uint8_t* sbuf0 = stage + e * 2 * T::kStageBuf;
+      int ti = 0, nst = 0;
+      for (int tile = tile0; tile < p.tiles; tile += tstep, ++ti) {
+        const int b = ti & 1;
+        const int n0 = (tile % p.tiles_n) * kTileN;
+        const int m0 = (tile / p.tiles_n) * p.BN;
+        const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
+        if constexpr (KIND == kW8A8) {
+          named_bar(1, nep);  // the previous tile's readers of sxs are done
+          for (int j = te; j < p.BN; j += nep) sxs[j] = (m0 + j < p.M) ? __ldg(p.sx + m0 + j) : 0.0f;
+          named_bar(1, nep);
+        }
+        bool ok = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 8);
+        ok = __all_sync(0xffffffffu, ok);  // warp-uniform before .sync.aligned TMEM loads
+        if (!ok) continue;  // keep taking part in the named barriers of later tiles
+        tc_fence_after();
+        const int nchunk = p.BN / 16;
+        if (cgrp >= nchunk) {  // no chunk for this warp: release buffer b at once
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + b);
+        }
+        for (int c = cgrp; c < nchunk; c += cstep) {
+          uint32_t r[16];
+          tmem_ld16(tmem_base + lane_off + b * kAccCols + c * 16, r);
+          tmem_ld_wait();
+          if (c + cstep >= nchunk) {
+            // this warp's last TMEM read of buffer b: the tile after next may reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + b);
+          }
+          uint8_t* sbuf = sbuf0 + (nst & 1) * T::kStageBuf;
+          if (lane == 0) bulk_wait_read<1>();  // the store that last used sbuf has read it
+          __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          v[c] = *reinterpret_cast<const uint4*>(src + sw128(t, c));
-        uint4 sc = make_uint4(0, 0, 0, 0);
-        if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
-        mbar_arrive(raw_empty + s);
-        constexpr int kHalves = T::kKbPerUnit;  // A tiles produced per raw stage
-#pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          const int sa = ia % p.n_a;
-          if (!(ok = mbar_wait(a_empty + sa, ((ia / p.n_a) & 1) ^ 1, abort_flag, 7))) break;
-          uint8_t* dst = abuf + sa * kATile;
-          if constexpr (KIND == kQ8) {
-            // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              const uint4 w = v[4 * h + cc];
-              uint4 o0, o1;
-              i8x4_to_h(w.x, o0.x, o0.y);
-              i8x4_to_h(w.y, o0.z, o0.w);
-              i8x4_to_h(w.z, o1.x, o1.y);
-              i8x4_to_h(w.w, o1.z, o1.w);
-              *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc)) = o0;
-              *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc + 1)) = o1;
-            }
-          } else {
-            // raw chunks 2h, 2h+1 (one 32-k group each) -> fp16 chunks 0..7
-            const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const int c = 2 * h + g;
-              const uint32_t spair = scw[c >> 1];
-              const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
-              const uint4 w = v[c];
-              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 0)) = nib8_to_h(w.x, s2);
-              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 1)) = nib8_to_h(w.y, s2);
-              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 2)) = nib8_to_h(w.z, s2);
-              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 3)) = nib8_to_h(w.w, s2);
+          for (int i = 0; i < 16; ++i) {
+            if constexpr (KIND == kS32) {
+              reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
+            } else if constexpr (KIND == kW8A8) {
+              reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+                  epi_w8a8(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc);
+            } else {
+              reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
             }
           }
           fence_proxy_async_smem();
-          mbar_arrive(a_full + sa);
-          ++ia;
-        }
-      }
-    }
-    // ----------------------------------------------------------- epilogue
-    ok = mbar_wait(acc_full, 0, abort_flag, 8);
-    ok = __all_sync(0xffffffffu, ok);  // warp-uniform before .sync.aligned TMEM loads
-    tc_fence_after();
-    const uint32_t trow = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int n = n0 + t;
-    if (p.splits == 1) {
-      if (ok) {
-        for (int cb = 0; cb < p.BN / 16; ++cb) {
-          uint32_t r[16];
-          tmem_ld16(trow + cb * 16, r);
-          tmem_ld_wait();
-          if (n < p.N) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int m = m0 + cb * 16 + i;
-              if (m < p.M) {
-                if constexpr (KIND == kS32)
-                  reinterpret_cast<int32_t*>(p.Y)[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[i]);
-                else
-                  reinterpret_cast<__half*>(p.Y)[static_cast<int64_t>(m) * p.N + n] = epi_value<KIND>(r[i], m, n, p);
-              }
-            }
+          __syncwarp();
+          const int nb = n0 + (warp & 3) * 32, mb = m0 + c * 16;
+          if (lane == 0 && nb < p.N && mb < p.M) {
+            tma_store_2d(&tmY, sbuf, nb, mb);  // rows >= M and columns >= N are clipped
+            bulk_commit();
           }
+          ++nst;
         }
       }
+      if (lane == 0) bulk_wait_all();
     } else {
-      // partial tile -> own shared memory, red[m_local][128] (32-bit words)
+      // split-K: one tile per CTA; partial tile -> own shared memory,
+      // red[m_local][128] (32-bit words), reduced below across the cluster
+      bool ok = mbar_wait(acc_full, 0, abort_flag, 8);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
       fence_proxy_async_smem();
       uint32_t* red = reinterpret_cast<uint32_t*>(smem);
-      for (int cb = 0; cb < p.BN / 16; ++cb) {
+      for (int c = cgrp; c < p.BN / 16; c += cstep) {
         uint32_t r[16];
-        tmem_ld16(trow + cb * 16, r);
+        tmem_ld16(tmem_base + lane_off + c * 16, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) red[(cb * 16 + i) * 128 + t] = ok ? r[i] : 0u;
+        for (int i = 0; i < 16; ++i) red[(c * 16 + i) * 128 + t] = ok ? r[i] : 0u;
       }
     }
   }
 
   // ------------------------------------------- split-K: cluster reduction
-  if (p.splits > 1) {
+  // CTA rank r reduces token rows [BN*r/S, BN*(r+1)/S) of the tile, summing
+  // the S partial tiles in rank order. Thread te owns 4 consecutive output
+  // channels (fixed for the whole loop, so their constants load once) and
+  // walks the rows with a stride of (epilogue threads / 32).
+  if (split) {
     __syncwarp();
     cluster_sync();
-    if (warp >= 4) {
-      const int t = threadIdx.x - 128;
+    if (warp >= 4 && !(T::kDequant && warp >= 8)) {
+      const int te = threadIdx.x - 128;
+      const int nep = T::kEpiWarps * 32;
+      const int n0 = (tile0 % p.tiles_n) * kTileN;
+      const int m0 = (tile0 / p.tiles_n) * p.BN;
       const int mb = p.BN * rank / p.splits, me = p.BN * (rank + 1) / p.splits;
+      const int nl = (te & 31) * 4;
+      const int n = n0 + nl;
+      RowConst<KIND> rc[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) rc[j] = row_const<KIND>(n + j, p);
       const uint32_t red_u32 = smem_u32(smem);
-      const int items = (me - mb) * 32;
-      for (int it = t; it < items; it += 128) {
-        const int ml = mb + (it >> 5);
-        const int nl = (it & 31) * 4;
-        const uint32_t off = red_u32 + static_cast<uint32_t>((ml * 128 + nl) * 4);
-        uint4 acc = ld_dsmem_v4(mapa_shared(off, 0));
-        for (int q = 1; q < p.splits; ++q) {
-          const uint4 v = ld_dsmem_v4(mapa_shared(off, q));
-          acc.x = reduce_add<KIND>(acc.x, v.x);
-          acc.y = reduce_add<KIND>(acc.y, v.y);
-          acc.z = reduce_add<KIND>(acc.z, v.z);
-          acc.w = reduce_add<KIND>(acc.w, v.w);
+      uint32_t peer[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) peer[q] = q < p.splits ? mapa_shared(red_u32, q) : 0u;
+      for (int ml = mb + (te >> 5); ml < me; ml += nep / 32) {
+        const uint32_t off = static_cast<uint32_t>((ml * 128 + nl) * 4);
+        uint4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < p.splits) v[q] = ld_dsmem_v4(peer[q] + off);
+        uint4 acc = v[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          if (q < p.splits) {
+            acc.x = reduce_add<KIND>(acc.x, v[q].x);
+            acc.y = reduce_add<KIND>(acc.y, v[q].y);
+            acc.z = reduce_add<KIND>(acc.z, v[q].z);
+            acc.w = reduce_add<KIND>(acc.w, v[q].w);
+          }
         }
-        const int m = m0 + ml, n = n0 + nl;
+        const int m = m0 + ml;
         if (m < p.M && n < p.N) {  // N % 16 == 0: all four columns are in range
           const int64_t o = static_cast<int64_t>(m) * p.N + n;
           if constexpr (KIND == kS32) {
             *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.Y) + o) = acc;
           } else {
-            __half h[4] = {epi_value<KIND>(acc.x, m, n, p), epi_value<KIND>(acc.y, m, n + 1, p),
-                           epi_value<KIND>(acc.z, m, n + 2, p), epi_value<KIND>(acc.w, m, n + 3, p)};
+            const uint32_t a4[4] = {acc.x, acc.y, acc.z, acc.w};
+            float sxm = 0.0f;
+            if constexpr (KIND == kW8A8) sxm = __ldg(p.sx + m);
+            __half h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if constexpr (KIND == kW8A8)
+                h[j] = epi_w8a8(static_cast<int32_t>(a4[j]), sxm, rc[j]);
+              else
+                h[j] = epi_wo<KIND>(__uint_as_float(a4[j]), rc[j]);
+            }
             *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.Y) + o) = *reinterpret_cast<uint2*>(h);
           }
         }
@@ -421,14 +636,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int i = (issued_x > p.n_x ? issued_x - p.n_x : 0); i < issued_x; ++i)
         mbar_wait_drain(x_full + (i % p.n_x), (i / p.n_x) & 1);
     } else if (warp == 1) {
-      mbar_wait_drain(acc_full, 0);  // MMAs issued before the abort have finished
+      umma_commit(mma_drain);  // MMAs issued before the abort finish before TMEM is freed
+      mbar_wait_drain(mma_drain, 0);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    tmem_dealloc(tmem_base, 2 * kAccCols);
   }
 }
 

@@ -11,6 +11,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace aria {
 
 constexpr int kRowThreads = 256;
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half*
                                                                    int K, int8_t* __restrict__ Q,
                                                                    float* __restrict__ S) {
   __shared__ float warp_max[kRowThreads / 32];
+  pdl_wait();  // X may be written by the preceding kernel
+  pdl_launch_dependents();
   const int64_t r = blockIdx.x;
   const int nchunk = K >> 3;
   const uint4* xr = reinterpret_cast<const uint4*>(X + r * static_cast<int64_t>(K));
@@ -98,6 +102,8 @@ __global__ void __launch_bounds__(256) pack_q4_kernel(const __half* __restrict__
                                                       int64_t nchunk,
                                                       uint32_t* __restrict__ P,
                                                       __half* __restrict__ S) {
+  pdl_wait();
+  pdl_launch_dependents();
   const uint4* w4 = reinterpret_cast<const uint4*>(W);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x; base < nchunk;
