@@ -48,6 +48,33 @@ WORKLOAD = ("layer-sequence replay: 24 blocks x {qkv 1536->4608, out 1536->1536,
 
 # ----------------------------------------------------------------- helpers --
 
+def kernel_source_sha256():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "int8_int4_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel, alg_bytes_per_launch):
+    """DRAM bytes per launch from the committed ncu record, scaled from the
+    captured case to this launch's algorithmic bytes; None if the kernel
+    sources changed since the counters were taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.json")) as f:
+            rec = json.load(f)
+        if rec["source_sha256"] != kernel_source_sha256():
+            return None, "stale: kernel changed since the ncu capture"
+        k = rec["kernels"][kernel]
+        return (k["dram_bytes"] * alg_bytes_per_launch / k["algorithmic_bytes"],
+                f"ncu capture of {k['case']} ({k['dram_bytes']} B DRAM for {k['algorithmic_bytes']} B "
+                f"algorithmic), scaled to this launch's algorithmic bytes")
+    except Exception as e:  # no record
+        return None, f"unavailable ({type(e).__name__})"
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -402,9 +429,9 @@ def run_ours(args, ws, rank):
     else:
         roof = {"bound": "hbm", "achieved": byt_l / t_l / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
     roof["kernel"] = {"q8": "qgemm_kernel<Q8>", "q4": "qgemm_kernel<Q4>", "w8a8_gemm": "qgemm_kernel<W8A8>",
                       "act_quant": "row_quant_i8_kernel"}[dom]
+    roof["traffic"], roof["traffic_source"] = measured_traffic(roof["kernel"], acct[dom][1] / launches)
     roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json "
                            + ("bf16_tflops_sustained" if roof["bound"] == "tensor" else "hbm_gbs")
                            + (" x 2 (nominal int8:fp16)" if dom == "w8a8_gemm" else ""))

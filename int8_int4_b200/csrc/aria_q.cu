@@ -140,20 +140,24 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.raw_stage = kind == kQ8 ? kATile : (kind == kQ4 ? kATile + kQ4ScaleTile : 0);
   p.raw_stage = (p.raw_stage + 1023u) & ~1023u;
   const int64_t budget = static_cast<int64_t>(di.smem_optin) - 1024 - 512 - stage_bytes - sxd_bytes;
+  // stage ring: one A tile + one X tile per stage (one MMA commit each);
+  // q8/q4 also keep a ring of raw packed weight tiles for the dequant warps
   int nr = 0, na = 0, nx = 0;
-  if (dq) {
-    na = bn > 128 ? 3 : 4;
-    for (int k = 8; k >= 2; --k) {
-      const int64_t need = static_cast<int64_t>(k) * p.raw_stage + na * kATile + k * p.x_stage;
-      if (need <= budget) { nr = nx = k; break; }
+  const int64_t st_bytes = kATile + p.x_stage;
+  for (int k = 8; k >= 2 && na == 0; --k) {
+    if (!dq) {
+      if (k * st_bytes <= budget) na = k;
+      continue;
     }
-    if (nr == 0) return fail(ARIA_ERR_UNSUPPORTED, "tile does not fit in shared memory");
-  } else {
-    for (int k = 8; k >= 2; --k) {
-      if (static_cast<int64_t>(k) * (kATile + p.x_stage) <= budget) { na = nx = k; break; }
-    }
-    if (na == 0) return fail(ARIA_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+    for (int r = 4; r >= 2; --r)
+      if (k * st_bytes + static_cast<int64_t>(r) * p.raw_stage <= budget) {
+        na = k;
+        nr = r;
+        break;
+      }
   }
+  if (na == 0) return fail(ARIA_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+  nx = na;
   p.n_raw = nr;
   p.n_a = na;
   p.n_x = nx;
@@ -163,7 +167,8 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.off_stage = p.off_x + nx * p.x_stage;
   p.off_sxd = p.off_stage + stage_bytes;
   p.off_bar = p.off_sxd + sxd_bytes;
-  if (static_cast<uint32_t>(bn) * 512u > p.off_stage) p.splits = splits = 1;  // no room to reduce
+  // the split-K partial tile (BN rows x 512 B) overlays the stage rings
+  if (static_cast<uint32_t>(bn) * 512u > p.off_stage) p.splits = splits = 1;
   const uint32_t nbar = 2 * (nr + na + nx) + 5;
   const size_t smem = 1024 + p.off_bar + nbar * 8 + 16;
   if (smem > static_cast<size_t>(di.smem_optin)) return fail(ARIA_ERR_UNSUPPORTED, "shared memory plan too large");
@@ -224,7 +229,7 @@ int max_clusters(int size, int threads, size_t smem) {
 
 template <int KIND>
 aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap& ts,
-                        const CUtensorMap& tx, const CUtensorMap& ty, cudaStream_t st) {
+                        const CUtensorMap& tx, cudaStream_t st) {
   auto kfn = aria::qgemm_kernel<KIND>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
@@ -253,7 +258,7 @@ aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap
     cfg.attrs = attr;
   }
   set_pdl(cfg, attr);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, ty, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, prm);
   if (e != cudaSuccess) return cuda_fail(e, "qgemm launch");
   return ARIA_OK;
 }
@@ -387,17 +392,6 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
     if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, bn,
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   }
-  CUtensorMap ty;
-  std::memset(&ty, 0, sizeof(ty));
-  if (pl.p.splits == 1) {
-    if (kind == kS32) {
-      if ((s = make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, M, N, 32, kEpiRows,
-                        CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
-    } else {
-      if ((s = make_map(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, N, 32, kEpiRows,
-                        CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
-    }
-  }
   pl.p.sw = static_cast<const float*>(kind == kQ4 ? nullptr : scales);
   pl.p.sx = sx;
   pl.p.bias = static_cast<const __half*>(bias);
@@ -406,10 +400,10 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
   pl.p.Y = Y;
   if (!pl.p.steer) pl.p.alpha = 0.0f;
   switch (kind) {
-    case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, ty, st);
-    case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, ty, st);
-    case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, ty, st);
-    case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, ty, st);
+    case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, st);
+    case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, st);
+    case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, st);
+    case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, st);
   }
   return fail(ARIA_ERR_INVALID_ARG, "unknown kind");
 }
@@ -460,3 +454,14 @@ ARIA_API aria_status aria_device_status(void* stream) {
   }
   return ARIA_OK;
 }
+
+#ifdef ARIA_TRACE
+// trace builds only: copy the per-CTA phase stamps to host memory
+ARIA_API int aria_trace_read(void* host, size_t bytes) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, aria::g_trace, bytes));
+}
+ARIA_API int aria_trace_clear(void) {
+  static long long zero[8192 * 16];
+  return static_cast<int>(cudaMemcpyToSymbol(aria::g_trace, zero, sizeof(zero)));
+}
+#endif

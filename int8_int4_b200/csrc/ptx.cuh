@@ -17,6 +17,24 @@ __device__ unsigned int g_status;
 __device__ unsigned int g_wait_site;
 
 constexpr unsigned kStatusTimeout = 1u;
+
+// Optional phase tracing (compile with -DARIA_TRACE): per-CTA %globaltimer
+// stamps of pipeline milestones, read back with aria_trace_read(). Compiled
+// out otherwise.
+#ifdef ARIA_TRACE
+__device__ long long g_trace[8192][16];
+#define ARIA_STAMP(slot)                                                                   \
+  do {                                                                                     \
+    const int cta_ = ((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) & 8191; \
+    long long t_;                                                                          \
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                 \
+    g_trace[cta_][(slot)] = t_;                                                            \
+  } while (0)
+#else
+#define ARIA_STAMP(slot) \
+  do {                   \
+  } while (0)
+#endif
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -310,6 +328,26 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t c0
                    reinterpret_cast<uint64_t>(m)),
                "r"(c0), "r"(c1)
                : "memory");
+}
+
+}  // namespace aria
+
+namespace aria {
+
+// store to distributed shared memory (an address from mapa_shared)
+__device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+}  // namespace aria
+
+namespace aria {
+
+// 32 lanes x 32 bits, one column per thread
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr) : "memory");
+  return r;
 }
 
 }  // namespace aria

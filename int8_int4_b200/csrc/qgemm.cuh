@@ -17,8 +17,9 @@
 //                tcgen05.mma issuer
 //   warp 2       TMA producer of activation tiles
 //   warps 4..7   epilogue: TMEM -> registers -> scale, bias, steer -> fp16 ->
-//                shared staging -> TMA bulk store; overlaps the next tile's
-//                mainloop through the second accumulator buffer
+//                transposed through shared memory -> coalesced 16-byte stores;
+//                overlaps the next tile's mainloop through the second
+//                accumulator buffer (W8A8 uses warps 8..11 for it as well)
 //   warps 8..11  q8/q4 only: dequantise raw weights into fp16 A tiles (one
 //                weight row per thread; exact int8 -> fp16; fp16 code*scale for q4)
 // Rings of shared-memory stages with mbarriers connect the roles; every wait
@@ -42,6 +43,7 @@ constexpr uint32_t kATile = 16384;       // 128 rows x 128 bytes
 constexpr uint32_t kQ4ScaleTile = 2048;  // 128 rows x 8 fp16 scales
 constexpr uint32_t kAccCols = 256;       // TMEM columns per accumulator buffer
 constexpr int kEpiRows = 16;             // tokens per epilogue store box
+constexpr int kL2Ahead = 4;              // weight units prefetched into L2 ahead of the TMA loads
 
 struct GemmParams {
   int M, N, K;
@@ -49,7 +51,7 @@ struct GemmParams {
   int units;              // K units: 128 (q8, W8A8) or 256 (q4) elements
   int splits;             // CTAs per cluster along K (1 = persistent over tiles)
   int tiles_n, tiles;     // weight-row tiles, total output tiles
-  int n_raw, n_a, n_x;    // ring depths
+  int n_raw, n_a, n_x;    // ring depths (raw packed weights; stages of A + X; n_x == n_a)
   uint32_t off_raw, off_a, off_x, off_stage, off_sxd, off_bar;
   uint32_t raw_stage, x_stage;
   const float* sw;        // per-channel weight scale (q8, W8A8)
@@ -150,12 +152,13 @@ __device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) 
 
 // W8A8 reference sequence: ((acc * s_x) * s_w) + bias + alpha*v in fp64, each
 // step rounded once (no contraction), then one rounding to fp16.
-__device__ __noinline__ __half epi_w8a8_fp64(int32_t acc, float sx, const RowConst<kW8A8>& c) {
+__device__ __noinline__ __half epi_w8a8_fp64(int32_t acc, float sx, float sw, float bias, float alpha,
+                                             float v, bool has_bias, bool has_steer) {
   double t = __dmul_rn(__dmul_rn(static_cast<double>(acc), static_cast<double>(sx)),
-                       static_cast<double>(c.sw));
-  if (c.has_bias) t = __dadd_rn(t, static_cast<double>(c.bias));
-  if (c.has_steer)  // a product of two fp32 values is exact in fp64
-    t = __dadd_rn(t, __dmul_rn(static_cast<double>(c.alpha), static_cast<double>(c.v)));
+                       static_cast<double>(sw));
+  if (has_bias) t = __dadd_rn(t, static_cast<double>(bias));
+  if (has_steer)  // a product of two fp32 values is exact in fp64
+    t = __dadd_rn(t, __dmul_rn(static_cast<double>(alpha), static_cast<double>(v)));
   return __double2half(t);
 }
 
@@ -174,9 +177,18 @@ __device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
 // values, where the sign of yl decides. The result equals the fp64
 // reference except if E lies within ~2^-46 of an fp16 midpoint (both are
 // then within one fp16 ulp). |acc| >= 2^22 takes the fp64 sequence.
-__device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst<kW8A8>& c) {
-  if (acc <= -(1 << 22) || acc >= (1 << 22)) return epi_w8a8_fp64(acc, sx, c);
-  const float a = __fsub_rn(__int_as_float(acc + 0x4B400000), 12582912.0f);  // exact int -> float
+//
+// w8a8_round() is the straight-line common path: it returns RN16(yh) and
+// sets `rare` when the result may need the midpoint fix-up (or the fp64
+// path), which w8a8_fixup() then applies. Keeping the common path free of
+// branches lets a chunk of elements be evaluated interleaved.
+struct W8A8Val {
+  float yh, yl;
+};
+
+__device__ __forceinline__ __half w8a8_round(int32_t acc, float sx, const RowConst<kW8A8>& c,
+                                             W8A8Val& v, bool& rare) {
+  const float a = __fsub_rn(__int_as_float(acc + 0x4B400000), 12582912.0f);  // exact if |acc| < 2^22
   const float ph = __fmul_rn(sx, c.sw);
   const float pl = __fmaf_rn(sx, c.sw, -ph);        // sx*sw == ph + pl
   float yh = __fmul_rn(a, ph);
@@ -194,12 +206,27 @@ __device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst
   const float s = __fadd_rn(yh, yl);                // renormalise: |yl| <= ulp(yh)/2
   yl = __fsub_rn(yl, __fsub_rn(s, yh));
   yh = s;
-  __half h = __float2half_rn(yh);
+  v.yh = yh;
+  v.yl = yl;
+  // An fp32 value can sit exactly on an fp16 rounding midpoint only if the 13
+  // bits below fp16 precision read 1000000000000 (fp16-normal range), or if it
+  // lies in the fp16-subnormal range.
+  const uint32_t yb = __float_as_uint(yh) & 0x7FFFFFFFu;
+  rare = (yl != 0.0f && ((yb & 0x1FFFu) == 0x1000u || yb < 0x38800000u)) ||
+         acc <= -(1 << 22) || acc >= (1 << 22);
+  return __float2half_rn(yh);
+}
+
+__device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float sw, float bias,
+                                          float alpha, float v, bool has_bias, bool has_steer,
+                                          float yh, float yl) {
+  if (acc <= -(1 << 22) || acc >= (1 << 22))
+    return epi_w8a8_fp64(acc, sx, sw, bias, alpha, v, has_bias, has_steer);
   // midpoint case: |yh| exactly halfway between |h| and its neighbour
   const float ay = fabsf(yh);
   const float ar = fabsf(__half2float(h));
   const float d = __fsub_rn(ay, ar);                // exact (Sterbenz, or ar == 0)
-  if (d != 0.0f && yl != 0.0f && ar < 65504.0f) {
+  if (d != 0.0f && ar < 65504.0f) {
     const uint32_t hb = __half_as_ushort(h) & 0x7FFFu;
     float half_gap;
     if (hb < 0x0400u) {
@@ -218,6 +245,31 @@ __device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst
     }
   }
   return h;
+}
+
+// No bias and no steering: y = fl(fl(acc) * fl(s_x*s_w)) is within 2 fp32 ulps
+// of the exact product E (acc is exact in fp32 below 2^22), so RN16(y) ==
+// RN16(E) unless y's 13 bits below fp16 precision are within 3 of the
+// midpoint pattern 0x1000, or y is outside the fp16 normal range; those
+// (about 0.1 % of elements) are flagged `rare` for the exact path.
+__device__ __forceinline__ __half w8a8_round_plain(int32_t acc, float sx, float sw, bool& rare) {
+  const float a = __fsub_rn(__int_as_float(acc + 0x4B400000), 12582912.0f);  // exact if |acc| < 2^22
+  const float y = __fmul_rn(a, __fmul_rn(sx, sw));
+  const uint32_t yb = __float_as_uint(y) & 0x7FFFFFFFu;
+  const uint32_t low = yb & 0x1FFFu;
+  rare = (low - 0x0FFDu) <= 6u                              // |low - 0x1000| <= 3
+         || (yb - 0x38800000u) >= (0x477FF000u - 0x38800000u) // |y| < 2^-14 or |y| >= 65504 - 16
+         || static_cast<uint32_t>(acc + (1 << 22) - 1) >= static_cast<uint32_t>((1 << 23) - 1);
+  rare = rare && y != 0.0f;  // an exact zero rounds to itself
+  return __float2half_rn(y);
+}
+
+__device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst<kW8A8>& c) {
+  W8A8Val v;
+  bool rare;
+  const __half h = w8a8_round(acc, sx, c, v, rare);
+  if (!rare) return h;
+  return w8a8_fixup(h, acc, sx, c.sw, c.bias, c.alpha, c.v, c.has_bias, c.has_steer, v.yh, v.yl);
 }
 
 // q8 / q4: fp32, (acc * s_w) + bias, then + alpha*v[n] (one fma), one rounding to fp16
@@ -242,8 +294,7 @@ __device__ __forceinline__ uint32_t reduce_add(uint32_t a, uint32_t b) {
 template <int KIND>
 __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     qgemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
-                 const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-                 const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmX, const GemmParams p) {
   using T = KindTraits<KIND>;
   extern __shared__ uint8_t dyn_smem[];
   // 1024-byte alignment of the shared-window address (128-byte swizzle atoms)
@@ -252,6 +303,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) ARIA_STAMP(0);
   const bool split = p.splits > 1;
   const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
   const int tile0 = split ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
@@ -267,13 +319,13 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   uint8_t* stage = smem + p.off_stage;
   float* sxs = reinterpret_cast<float*>(smem + p.off_sxd);   // s_x of the current m-tile
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  // one stage = an A tile (weights, 128 rows x 128 B of K) and an X tile
+  // (activations, BN rows x 128 B of K); one commit releases both
   uint64_t* raw_full = bars;
   uint64_t* raw_empty = raw_full + p.n_raw;
-  uint64_t* a_full = raw_empty + p.n_raw;
-  uint64_t* a_empty = a_full + p.n_a;
-  uint64_t* x_full = a_empty + p.n_a;
-  uint64_t* x_empty = x_full + p.n_x;
-  uint64_t* acc_full = x_empty + p.n_x;   // [2]
+  uint64_t* st_full = raw_empty + p.n_raw;
+  uint64_t* st_empty = st_full + p.n_a;
+  uint64_t* acc_full = st_empty + p.n_a;  // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
   uint64_t* mma_drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
@@ -285,12 +337,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       mbar_init(raw_empty + i, 128);
     }
     for (int i = 0; i < p.n_a; ++i) {
-      mbar_init(a_full + i, T::kDequant ? 128 : 1);
-      mbar_init(a_empty + i, 1);
-    }
-    for (int i = 0; i < p.n_x; ++i) {
-      mbar_init(x_full + i, 1);
-      mbar_init(x_empty + i, 1);
+      // q8/q4: 128 dequant threads + the X producer; W8A8: the single producer
+      mbar_init(st_full + i, T::kDequant ? 129 : 1);
+      mbar_init(st_empty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full + i, 1);
@@ -304,7 +353,6 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
     if constexpr (KIND == kQ4) prefetch_tmap(&tmS);
-    if (!split) prefetch_tmap(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * kAccCols);
@@ -319,7 +367,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   // coherent), and the shared-memory loads below only start after the wait.
   if (warp == 0 && lane == 0 && tile0 < p.tiles) {
     const int n0 = (tile0 % p.tiles_n) * kTileN;
-    const int npf = nu < 4 ? nu : 4;
+    const int npf = nu < kL2Ahead ? nu : kL2Ahead;
     for (int i = 0; i < npf; ++i) {
       tma_prefetch_2d(&tmW, (u_begin + i) * 128, n0);
       if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
@@ -328,10 +376,14 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   // Inputs may come from the preceding kernel in the stream (programmatic
   // dependent launch): everything above overlapped its tail; nothing below
   // reads or writes global memory before it has completed.
+  if (threadIdx.x == 0) ARIA_STAMP(1);
   pdl_wait();
   pdl_launch_dependents();
+  if (threadIdx.x == 0) ARIA_STAMP(2);
 
   int issued_w = 0, issued_x = 0;  // kept for the teardown drain
+  bool epi_ok = true;               // split-K: this CTA's accumulator is complete
+  const bool epi_warp = warp >= 4 && !(T::kDequant && warp >= 8);
 
   if (warp == 0) {
     // ------------------------------------------------ weight tile producer
@@ -346,6 +398,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             if (!(ok = mbar_wait(raw_empty + s, ((issued_w / p.n_raw) & 1) ^ 1, abort_flag, 1))) break;
             uint8_t* dst = raw + s * p.raw_stage;
             const int u = u_begin + i;
+            if (i + kL2Ahead < nu) {  // keep the weight stream kL2Ahead units ahead in L2
+              tma_prefetch_2d(&tmW, (u + kL2Ahead) * 128, n0);
+              if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u + kL2Ahead) * 8, n0);
+            }
             if constexpr (KIND == kQ8) {
               mbar_arrive_expect_tx(raw_full + s, kATile);
               tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);
@@ -357,17 +413,21 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             ++issued_w;
           }
         } else {
+          const uint64_t polx = policy_evict_last();
+          const int m0 = (tile / p.tiles_n) * p.BN;
           for (int kb = 0; kb < nkb; ++kb) {
             const int s = issued_w % p.n_a;
-            if (!(ok = mbar_wait(a_empty + s, ((issued_w / p.n_a) & 1) ^ 1, abort_flag, 2))) break;
-            mbar_arrive_expect_tx(a_full + s, kATile);
-            tma_load_2d(&tmW, a_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
+            if (!(ok = mbar_wait(st_empty + s, ((issued_w / p.n_a) & 1) ^ 1, abort_flag, 2))) break;
+            if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * 128, n0);
+            mbar_arrive_expect_tx(st_full + s, kATile + p.x_stage);
+            tma_load_2d(&tmW, st_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
+            tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * 128, m0, polx);
             ++issued_w;
           }
         }
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 && T::kDequant) {
     // -------------------------------------------- activation tile producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();   // re-read by every weight tile
@@ -376,10 +436,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
         const int m0 = (tile / p.tiles_n) * p.BN;
         for (int kb = 0; kb < nkb; ++kb) {
-          const int s = issued_x % p.n_x;
-          if (!(ok = mbar_wait(x_empty + s, ((issued_x / p.n_x) & 1) ^ 1, abort_flag, 3))) break;
-          mbar_arrive_expect_tx(x_full + s, p.x_stage);
-          tma_load_2d(&tmX, x_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
+          const int s = issued_x % p.n_a;
+          if (!(ok = mbar_wait(st_empty + s, ((issued_x / p.n_a) & 1) ^ 1, abort_flag, 3))) break;
+          mbar_arrive_expect_tx(st_full + s, p.x_stage);
+          tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
           ++issued_x;
         }
       }
@@ -393,13 +453,14 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
         const int b = ti & 1;
         if (!(ok = mbar_wait(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9))) break;
+        if (ti == 0) ARIA_STAMP(3);
         tc_fence_after();
         const uint32_t dt = tmem_base + b * kAccCols;
         for (int kb = 0; kb < nkb; ++kb, ++ka) {
-          const int sa = ka % p.n_a, sx = ka % p.n_x;
-          ok = mbar_wait(a_full + sa, (ka / p.n_a) & 1, abort_flag, 4) &&
-               mbar_wait(x_full + sx, (ka / p.n_x) & 1, abort_flag, 5);
+          const int sa = ka % p.n_a, sx = sa;
+          ok = mbar_wait(st_full + sa, (ka / p.n_a) & 1, abort_flag, 4);
           if (!ok) break;
+          if (ka == 0) ARIA_STAMP(4);
           tc_fence_after();
           const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
           const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sx * p.x_stage));
@@ -410,10 +471,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             else
               umma_i8(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
           }
-          umma_commit(a_empty + sa);
-          umma_commit(x_empty + sx);
+          umma_commit(st_empty + sa);  // releases both tiles of the stage
         }
         umma_commit(acc_full + b);  // also fires when nothing was issued
+        ARIA_STAMP(5);
       }
     }
   } else if (T::kDequant && warp >= 8) {
@@ -426,6 +487,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         for (int i = 0; i < nu && ok; ++i, ++ir) {
           const int s = ir % p.n_raw;
           if (!(ok = mbar_wait(raw_full + s, (ir / p.n_raw) & 1, abort_flag, 6))) break;
+          if (t == 0 && ir == 0) ARIA_STAMP(12);
           const uint8_t* src = raw + s * p.raw_stage;
           uint4 v[8];
 #pragma unroll
@@ -436,7 +498,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 #pragma unroll
           for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
             const int sa = ia % p.n_a;
-            if (!(ok = mbar_wait(a_empty + sa, ((ia / p.n_a) & 1) ^ 1, abort_flag, 7))) break;
+            if (!(ok = mbar_wait(st_empty + sa, ((ia / p.n_a) & 1) ^ 1, abort_flag, 7))) break;
             uint8_t* dst = abuf + sa * kATile;
             if constexpr (KIND == kQ8) {
               // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
@@ -467,7 +529,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
               }
             }
             fence_proxy_async_smem();
-            mbar_arrive(a_full + sa);
+            mbar_arrive(st_full + sa);
             ++ia;
           }
         }
@@ -499,6 +561,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         bool ok = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 8);
         ok = __all_sync(0xffffffffu, ok);  // warp-uniform before .sync.aligned TMEM loads
         if (!ok) continue;  // keep taking part in the named barriers of later tiles
+        if (te == 0 && ti == 0) ARIA_STAMP(6);
         tc_fence_after();
         const int nchunk = p.BN / 16;
         if (cgrp >= nchunk) {  // no chunk for this warp: release buffer b at once
@@ -510,66 +573,118 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           uint32_t r[16];
           tmem_ld16(tmem_base + lane_off + b * kAccCols + c * 16, r);
           tmem_ld_wait();
+          // transpose the warp's 32 channels x 16 tokens through shared memory
+          // ([16][32] box), then coalesced 16-byte stores along the channels
+          uint8_t* sbuf = sbuf0 + (nst & 1) * T::kStageBuf;
+          if constexpr (KIND == kW8A8) {
+            // common path, straight-line over the chunk; elements flagged rare
+            // are redone below from their accumulator, re-read from TMEM
+            uint32_t rare_mask = 0;
+            if (!rc.has_bias && !rc.has_steer) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                bool rare;
+                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+                    w8a8_round_plain(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc.sw, rare);
+                rare_mask |= static_cast<uint32_t>(rare) << i;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                bool rare;
+                W8A8Val vv;
+                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+                    w8a8_round(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc, vv, rare);
+                rare_mask |= static_cast<uint32_t>(rare) << i;
+              }
+            }
+            uint32_t any = __reduce_or_sync(0xffffffffu, rare_mask);
+            while (any) {  // warp-uniform loop: the TMEM load is .sync.aligned
+              const int i = __ffs(any) - 1;
+              any &= any - 1;
+              const uint32_t a1 = tmem_ld1(tmem_base + lane_off + b * kAccCols + c * 16 + i);
+              tmem_ld_wait();
+              if (rare_mask & (1u << i)) {
+                const float sxi = sxs[c * 16 + i];
+                bool rare;
+                W8A8Val vv;
+                const __half h0 = w8a8_round(static_cast<int32_t>(a1), sxi, rc, vv, rare);
+                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+                    w8a8_fixup(h0, static_cast<int32_t>(a1), sxi, rc.sw, rc.bias, rc.alpha, rc.v,
+                               rc.has_bias, rc.has_steer, vv.yh, vv.yl);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if constexpr (KIND == kS32)
+                reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
+              else
+                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
+            }
+          }
           if (c + cstep >= nchunk) {
             // this warp's last TMEM read of buffer b: the tile after next may reuse it
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty + b);
           }
-          uint8_t* sbuf = sbuf0 + (nst & 1) * T::kStageBuf;
-          if (lane == 0) bulk_wait_read<1>();  // the store that last used sbuf has read it
           __syncwarp();
+          {
+            constexpr int kRowChunks = 32 * T::kOutBytes / 16;     // 16-byte chunks per box row
+            constexpr int kPerLane = 16 * kRowChunks / 32;
+            const int nb = n0 + (warp & 3) * 32;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if constexpr (KIND == kS32) {
-              reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
-            } else if constexpr (KIND == kW8A8) {
-              reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-                  epi_w8a8(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc);
-            } else {
-              reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
+            for (int j = 0; j < kPerLane; ++j) {
+              const int idx = j * 32 + lane;
+              const int row = idx / kRowChunks, ch = idx % kRowChunks;
+              const int m = m0 + c * 16 + row;
+              const int n = nb + ch * (16 / static_cast<int>(T::kOutBytes));
+              const uint4 v = *reinterpret_cast<const uint4*>(sbuf + row * 32 * T::kOutBytes + ch * 16);
+              if (m < p.M && n < p.N)  // N % 16 == 0: a 16-byte chunk is wholly in or out
+                *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Y) +
+                                          (static_cast<int64_t>(m) * p.N + n) * T::kOutBytes) = v;
             }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          const int nb = n0 + (warp & 3) * 32, mb = m0 + c * 16;
-          if (lane == 0 && nb < p.N && mb < p.M) {
-            tma_store_2d(&tmY, sbuf, nb, mb);  // rows >= M and columns >= N are clipped
-            bulk_commit();
           }
           ++nst;
         }
+        if (te == 0) ARIA_STAMP(7);
       }
-      if (lane == 0) bulk_wait_all();
     } else {
-      // split-K: one tile per CTA; partial tile -> own shared memory,
-      // red[m_local][128] (32-bit words), reduced below across the cluster
+      // split-K: one tile per CTA; wait for its partial accumulator
       bool ok = mbar_wait(acc_full, 0, abort_flag, 8);
-      ok = __all_sync(0xffffffffu, ok);
+      epi_ok = __all_sync(0xffffffffu, ok);
+    }
+  }
+
+  // ------------------------------------------- split-K: cluster reduction
+  // Each CTA first writes its partial tile to its own shared memory,
+  // red[m_local][128] (32-bit words, overlaying the now idle stage rings).
+  // After a cluster barrier, rank r reduces token rows [BN*r/S, BN*(r+1)/S),
+  // summing the S partials in rank order (deterministic) with
+  // distributed-shared-memory loads, four rows in flight per thread.
+  if (split) {
+    if (epi_warp) {
+      const int e = warp - 4;
+      const int t = (warp & 3) * 32 + lane;
+      const int cgrp = e >> 2, cstep = T::kEpiWarps >> 2;
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
       tc_fence_after();
-      fence_proxy_async_smem();
       uint32_t* red = reinterpret_cast<uint32_t*>(smem);
       for (int c = cgrp; c < p.BN / 16; c += cstep) {
         uint32_t r[16];
         tmem_ld16(tmem_base + lane_off + c * 16, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) red[(c * 16 + i) * 128 + t] = ok ? r[i] : 0u;
+        for (int i = 0; i < 16; ++i) red[(c * 16 + i) * 128 + t] = epi_ok ? r[i] : 0u;
       }
     }
-  }
-
-  // ------------------------------------------- split-K: cluster reduction
-  // CTA rank r reduces token rows [BN*r/S, BN*(r+1)/S) of the tile, summing
-  // the S partial tiles in rank order. Thread te owns 4 consecutive output
-  // channels (fixed for the whole loop, so their constants load once) and
-  // walks the rows with a stride of (epilogue threads / 32).
-  if (split) {
     __syncwarp();
     cluster_sync();
-    if (warp >= 4 && !(T::kDequant && warp >= 8)) {
+    ARIA_STAMP(8);
+    if (epi_warp) {
       const int te = threadIdx.x - 128;
-      const int nep = T::kEpiWarps * 32;
+      const int rstep = T::kEpiWarps;  // rows advanced per pass (32 threads per row)
       const int n0 = (tile0 % p.tiles_n) * kTileN;
       const int m0 = (tile0 / p.tiles_n) * p.BN;
       const int mb = p.BN * rank / p.splits, me = p.BN * (rank + 1) / p.splits;
@@ -579,62 +694,76 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) rc[j] = row_const<KIND>(n + j, p);
       const uint32_t red_u32 = smem_u32(smem);
-      uint32_t peer[8];
+      constexpr int kRows = 4;
+      for (int ml0 = mb + (te >> 5); ml0 < me; ml0 += kRows * rstep) {
+        uint4 acc[kRows];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) peer[q] = q < p.splits ? mapa_shared(red_u32, q) : 0u;
-      for (int ml = mb + (te >> 5); ml < me; ml += nep / 32) {
-        const uint32_t off = static_cast<uint32_t>((ml * 128 + nl) * 4);
-        uint4 v[8];
+        for (int u = 0; u < kRows; ++u) acc[u] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < p.splits; ++q) {
+          uint4 v[kRows];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < p.splits) v[q] = ld_dsmem_v4(peer[q] + off);
-        uint4 acc = v[0];
+          for (int u = 0; u < kRows; ++u) {
+            const int ml = ml0 + u * rstep;
+            if (ml < me)
+              v[u] = ld_dsmem_v4(mapa_shared(red_u32 + static_cast<uint32_t>((ml * 128 + nl) * 4), q));
+          }
 #pragma unroll
-        for (int q = 1; q < 8; ++q) {
-          if (q < p.splits) {
-            acc.x = reduce_add<KIND>(acc.x, v[q].x);
-            acc.y = reduce_add<KIND>(acc.y, v[q].y);
-            acc.z = reduce_add<KIND>(acc.z, v[q].z);
-            acc.w = reduce_add<KIND>(acc.w, v[q].w);
+          for (int u = 0; u < kRows; ++u) {
+            if (q == 0) {
+              acc[u] = v[u];
+            } else {
+              acc[u].x = reduce_add<KIND>(acc[u].x, v[u].x);
+              acc[u].y = reduce_add<KIND>(acc[u].y, v[u].y);
+              acc[u].z = reduce_add<KIND>(acc[u].z, v[u].z);
+              acc[u].w = reduce_add<KIND>(acc[u].w, v[u].w);
+            }
           }
         }
-        const int m = m0 + ml;
-        if (m < p.M && n < p.N) {  // N % 16 == 0: all four columns are in range
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) {
+          const int ml = ml0 + u * rstep;
+          const int m = m0 + ml;
+          if (ml >= me || m >= p.M || n >= p.N) continue;  // N % 16 == 0: 4 columns in range
           const int64_t o = static_cast<int64_t>(m) * p.N + n;
           if constexpr (KIND == kS32) {
-            *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.Y) + o) = acc;
+            *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.Y) + o) = acc[u];
           } else {
-            const uint32_t a4[4] = {acc.x, acc.y, acc.z, acc.w};
+            const uint32_t a4[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
             float sxm = 0.0f;
             if constexpr (KIND == kW8A8) sxm = __ldg(p.sx + m);
             __half h[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int k = 0; k < 4; ++k) {
               if constexpr (KIND == kW8A8)
-                h[j] = epi_w8a8(static_cast<int32_t>(a4[j]), sxm, rc[j]);
+                h[k] = epi_w8a8(static_cast<int32_t>(a4[k]), sxm, rc[k]);
               else
-                h[j] = epi_wo<KIND>(__uint_as_float(a4[j]), rc[j]);
+                h[k] = epi_wo<KIND>(__uint_as_float(a4[k]), rc[k]);
             }
             *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.Y) + o) = *reinterpret_cast<uint2*>(h);
           }
         }
       }
     }
+    ARIA_STAMP(9);
     __syncwarp();
     cluster_sync();
+    ARIA_STAMP(10);
   }
 
   // ---------------------------------------------------------------- teardown
   if (*abort_flag && lane == 0) {
     // drain copies still in flight into this CTA's shared memory
+    // (q8/q4 stage barriers also wait for dequant arrivals, so only the raw
+    // ring and W8A8 stages are drained here; X loads of q8/q4 stages were
+    // issued only after their stage was empty and complete on their own)
     if (warp == 0) {
       const int nring = T::kDequant ? p.n_raw : p.n_a;
-      uint64_t* full = T::kDequant ? raw_full : a_full;
+      uint64_t* full = T::kDequant ? raw_full : st_full;
       for (int i = (issued_w > nring ? issued_w - nring : 0); i < issued_w; ++i)
         mbar_wait_drain(full + (i % nring), (i / nring) & 1);
-    } else if (warp == 2) {
-      for (int i = (issued_x > p.n_x ? issued_x - p.n_x : 0); i < issued_x; ++i)
-        mbar_wait_drain(x_full + (i % p.n_x), (i / p.n_x) & 1);
+    } else if (warp == 2 && issued_x > 0) {
+      const uint64_t t0 = globaltimer();  // X loads of q8/q4: allow 100 us to land
+      while (globaltimer() - t0 < 100000ull) __nanosleep(1000);
     } else if (warp == 1) {
       umma_commit(mma_drain);  // MMAs issued before the abort finish before TMEM is freed
       mbar_wait_drain(mma_drain, 0);
@@ -646,6 +775,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * kAccCols);
   }
+  if (threadIdx.x == 0) ARIA_STAMP(11);
 }
 
 }  // namespace aria

@@ -137,6 +137,25 @@ def test_w8a8_within_one_ulp(M, N, K, bias, steer):
     assert d.max() <= 1, d.max()
 
 
+def test_w8a8_large_accumulators_take_exact_path():
+    """|acc| >= 2^22 (all codes +-127 over K = 4096) and exact fp16 results
+    exercise the kernel's fp64 branch; sign patterns vary per row/column."""
+    M, N, K = 64, 256, 4096
+    rng = np.random.default_rng(5)
+    sgn_x = rng.choice([-1.0, 1.0], (M, 1)) * np.ones((1, K))
+    sgn_w = rng.choice([-1.0, 1.0], (N, 1)) * np.ones((1, K))
+    sgn_x[:, ::3] *= -1                        # mixed signs inside a row
+    X = torch.from_numpy((sgn_x * rng.uniform(0.5, 2.0, (M, 1))).astype(np.float16))
+    W = torch.from_numpy((sgn_w * 0.01).astype(np.float16))
+    Wq, sw = aq.qpack("q8", W.cuda())
+    Xq, sx = aq.act_quant(X.cuda())
+    acc = aq.qgemm_s32(Xq, Wq).abs().max().item()
+    assert acc >= 2 ** 22
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx)
+    ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy())
+    assert np.array_equal(Y.cpu().numpy().view(np.uint16), ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(4096, 6144, 1536), (4096, 1536, 6144), (4096, 4608, 1536)])
 def test_w8a8_full_size_sampled(M, N, K):
     key = f"gpu/w8a8f/{M}x{N}x{K}"
@@ -146,6 +165,8 @@ def test_w8a8_full_size_sampled(M, N, K):
     ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(), rows=rows)
     d = ulp_dist(Y.cpu().numpy().view(np.uint16)[rows], ref)
     assert d.max() <= 1, d.max()
+    # the exact-rounding epilogue is expected to agree bit for bit
+    assert (d == 0).mean() == 1.0, (d != 0).sum()
 
 
 # ------------------------------------------------------- weight-only GEMM ---
