@@ -351,3 +351,13 @@ __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
 }
 
 }  // namespace aria
+
+namespace aria {
+
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+}  // namespace aria

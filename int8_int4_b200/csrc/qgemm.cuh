@@ -290,6 +290,91 @@ __device__ __forceinline__ uint32_t reduce_add(uint32_t a, uint32_t b) {
     return __float_as_uint(__uint_as_float(a) + __uint_as_float(b));
 }
 
+// Epilogue of one 16-column chunk for the calling warp, in two halves so the
+// caller can release the accumulator buffer between them.
+// compute: TMEM (row base `tacc` = this warp's 32 lanes of the buffer) ->
+// registers -> scale / bias / steer -> fp16 -> 32x16 box in `sbuf`.
+template <int KIND>
+__device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int lane, uint8_t* sbuf,
+                                                       const RowConst<KIND>& rc, const float* sxs) {
+    uint32_t r[16];
+    tmem_ld16(tacc + c * 16, r);
+    tmem_ld_wait();
+    // transpose the warp's 32 channels x 16 tokens through shared memory
+    // ([16][32] box), then coalesced 16-byte stores along the channels
+    if constexpr (KIND == kW8A8) {
+      // common path, straight-line over the chunk; elements flagged rare
+      // are redone below from their accumulator, re-read from TMEM
+      uint32_t rare_mask = 0;
+      if (!rc.has_bias && !rc.has_steer) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          bool rare;
+          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+              w8a8_round_plain(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc.sw, rare);
+          rare_mask |= static_cast<uint32_t>(rare) << i;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          bool rare;
+          W8A8Val vv;
+          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+              w8a8_round(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc, vv, rare);
+          rare_mask |= static_cast<uint32_t>(rare) << i;
+        }
+      }
+      uint32_t any = __reduce_or_sync(0xffffffffu, rare_mask);
+      while (any) {  // warp-uniform loop: the TMEM load is .sync.aligned
+        const int i = __ffs(any) - 1;
+        any &= any - 1;
+        const uint32_t a1 = tmem_ld1(tacc + c * 16 + i);
+        tmem_ld_wait();
+        if (rare_mask & (1u << i)) {
+          const float sxi = sxs[c * 16 + i];
+          bool rare;
+          W8A8Val vv;
+          const __half h0 = w8a8_round(static_cast<int32_t>(a1), sxi, rc, vv, rare);
+          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
+              w8a8_fixup(h0, static_cast<int32_t>(a1), sxi, rc.sw, rc.bias, rc.alpha, rc.v,
+                         rc.has_bias, rc.has_steer, vv.yh, vv.yl);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if constexpr (KIND == kS32)
+          reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
+        else
+          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
+      }
+    }
+}
+
+// store: the box in `sbuf`, transposed, as coalesced 16-byte stores of
+// channels [nb, nb + 32) x tokens [m0 + 16c, m0 + 16c + 16).
+template <int KIND>
+__device__ __forceinline__ void epilogue_chunk_store(int c, int nb, int m0, int lane, const uint8_t* sbuf,
+                                                     const GemmParams& p) {
+  using T = KindTraits<KIND>;
+    __syncwarp();
+    {
+      constexpr int kRowChunks = 32 * T::kOutBytes / 16;     // 16-byte chunks per box row
+      constexpr int kPerLane = 16 * kRowChunks / 32;
+#pragma unroll
+      for (int j = 0; j < kPerLane; ++j) {
+        const int idx = j * 32 + lane;
+        const int row = idx / kRowChunks, ch = idx % kRowChunks;
+        const int m = m0 + c * 16 + row;
+        const int n = nb + ch * (16 / static_cast<int>(T::kOutBytes));
+        const uint4 v = *reinterpret_cast<const uint4*>(sbuf + row * 32 * T::kOutBytes + ch * 16);
+        if (m < p.M && n < p.N)  // N % 16 == 0: a 16-byte chunk is wholly in or out
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Y) +
+                                    (static_cast<int64_t>(m) * p.N + n) * T::kOutBytes) = v;
+      }
+    }
+}
+
 // ------------------------------------------------------------------ kernel --
 template <int KIND>
 __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
@@ -534,6 +619,30 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           }
         }
       }
+      // The CTA's last tile: these warps take its odd epilogue chunks, with
+      // store boxes staged in the now idle raw-weight ring.
+      if (ok && !split && tile0 < p.tiles) {
+        const int ti = (p.tiles - tile0 + tstep - 1) / tstep - 1;
+        const int tile = tile0 + ti * tstep;
+        const int b = ti & 1;
+        const int n0 = (tile % p.tiles_n) * kTileN;
+        const int m0 = (tile / p.tiles_n) * p.BN;
+        const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
+        bool ok2 = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 10);
+        ok2 = __all_sync(0xffffffffu, ok2);
+        if (ok2) {
+          tc_fence_after();
+          const uint32_t tacc = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + b * kAccCols;
+          uint8_t* sb0 = raw + (warp - 8) * 2 * T::kStageBuf;
+          int nst = 0;
+          for (int c = 1; c < p.BN / 16; c += 2, ++nst) {
+            uint8_t* sbuf = sb0 + (nst & 1) * T::kStageBuf;
+            epilogue_chunk_compute<KIND>(c, tacc, lane, sbuf, rc, sxs);
+            __syncwarp();
+            epilogue_chunk_store<KIND>(c, n0 + (warp & 3) * 32, m0, lane, sbuf, p);
+          }
+        }
+      }
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- epilogue
@@ -564,88 +673,25 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         if (te == 0 && ti == 0) ARIA_STAMP(6);
         tc_fence_after();
         const int nchunk = p.BN / 16;
+        // q8/q4: the dequant warps have no work left during the CTA's last
+        // tile and take its odd chunks (see the end of the dequant role)
+        const int cs = (T::kDequant && tile + tstep >= p.tiles) ? 2 : cstep;
         if (cgrp >= nchunk) {  // no chunk for this warp: release buffer b at once
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty + b);
         }
-        for (int c = cgrp; c < nchunk; c += cstep) {
-          uint32_t r[16];
-          tmem_ld16(tmem_base + lane_off + b * kAccCols + c * 16, r);
-          tmem_ld_wait();
-          // transpose the warp's 32 channels x 16 tokens through shared memory
-          // ([16][32] box), then coalesced 16-byte stores along the channels
+        for (int c = cgrp; c < nchunk; c += cs) {
           uint8_t* sbuf = sbuf0 + (nst & 1) * T::kStageBuf;
-          if constexpr (KIND == kW8A8) {
-            // common path, straight-line over the chunk; elements flagged rare
-            // are redone below from their accumulator, re-read from TMEM
-            uint32_t rare_mask = 0;
-            if (!rc.has_bias && !rc.has_steer) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                bool rare;
-                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-                    w8a8_round_plain(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc.sw, rare);
-                rare_mask |= static_cast<uint32_t>(rare) << i;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                bool rare;
-                W8A8Val vv;
-                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-                    w8a8_round(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc, vv, rare);
-                rare_mask |= static_cast<uint32_t>(rare) << i;
-              }
-            }
-            uint32_t any = __reduce_or_sync(0xffffffffu, rare_mask);
-            while (any) {  // warp-uniform loop: the TMEM load is .sync.aligned
-              const int i = __ffs(any) - 1;
-              any &= any - 1;
-              const uint32_t a1 = tmem_ld1(tmem_base + lane_off + b * kAccCols + c * 16 + i);
-              tmem_ld_wait();
-              if (rare_mask & (1u << i)) {
-                const float sxi = sxs[c * 16 + i];
-                bool rare;
-                W8A8Val vv;
-                const __half h0 = w8a8_round(static_cast<int32_t>(a1), sxi, rc, vv, rare);
-                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-                    w8a8_fixup(h0, static_cast<int32_t>(a1), sxi, rc.sw, rc.bias, rc.alpha, rc.v,
-                               rc.has_bias, rc.has_steer, vv.yh, vv.yl);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if constexpr (KIND == kS32)
-                reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
-              else
-                reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
-            }
-          }
-          if (c + cstep >= nchunk) {
+          const uint32_t tacc = tmem_base + lane_off + b * kAccCols;
+          epilogue_chunk_compute<KIND>(c, tacc, lane, sbuf, rc, sxs);
+          if (c + cs >= nchunk) {
             // this warp's last TMEM read of buffer b: the tile after next may reuse it
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty + b);
           }
-          __syncwarp();
-          {
-            constexpr int kRowChunks = 32 * T::kOutBytes / 16;     // 16-byte chunks per box row
-            constexpr int kPerLane = 16 * kRowChunks / 32;
-            const int nb = n0 + (warp & 3) * 32;
-#pragma unroll
-            for (int j = 0; j < kPerLane; ++j) {
-              const int idx = j * 32 + lane;
-              const int row = idx / kRowChunks, ch = idx % kRowChunks;
-              const int m = m0 + c * 16 + row;
-              const int n = nb + ch * (16 / static_cast<int>(T::kOutBytes));
-              const uint4 v = *reinterpret_cast<const uint4*>(sbuf + row * 32 * T::kOutBytes + ch * 16);
-              if (m < p.M && n < p.N)  // N % 16 == 0: a 16-byte chunk is wholly in or out
-                *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Y) +
-                                          (static_cast<int64_t>(m) * p.N + n) * T::kOutBytes) = v;
-            }
-          }
+          epilogue_chunk_store<KIND>(c, n0 + (warp & 3) * 32, m0, lane, sbuf, p);
           ++nst;
         }
         if (te == 0) ARIA_STAMP(7);
@@ -719,6 +765,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             }
           }
         }
+        uint32_t rare_mask = 0;  // W8A8: elements to redo exactly (bit 4u+k)
 #pragma unroll
         for (int u = 0; u < kRows; ++u) {
           const int ml = ml0 + u * rstep;
@@ -729,17 +776,42 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.Y) + o) = acc[u];
           } else {
             const uint32_t a4[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
-            float sxm = 0.0f;
-            if constexpr (KIND == kW8A8) sxm = __ldg(p.sx + m);
             __half h[4];
+            if constexpr (KIND == kW8A8) {
+              const float sxm = __ldg(p.sx + m);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if constexpr (KIND == kW8A8)
-                h[k] = epi_w8a8(static_cast<int32_t>(a4[k]), sxm, rc[k]);
-              else
-                h[k] = epi_wo<KIND>(__uint_as_float(a4[k]), rc[k]);
+              for (int k = 0; k < 4; ++k) {
+                bool rare;
+                if (!rc[k].has_bias && !rc[k].has_steer) {
+                  h[k] = w8a8_round_plain(static_cast<int32_t>(a4[k]), sxm, rc[k].sw, rare);
+                } else {
+                  W8A8Val vv;
+                  h[k] = w8a8_round(static_cast<int32_t>(a4[k]), sxm, rc[k], vv, rare);
+                }
+                rare_mask |= static_cast<uint32_t>(rare) << (4 * u + k);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) h[k] = epi_wo<KIND>(__uint_as_float(a4[k]), rc[k]);
             }
             *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.Y) + o) = *reinterpret_cast<uint2*>(h);
+          }
+        }
+        if constexpr (KIND == kW8A8) {
+          // rare elements: re-sum the partials and round exactly; these later
+          // stores of the same thread replace the values written above
+          while (rare_mask) {
+            const int idx = __ffs(rare_mask) - 1;
+            rare_mask &= rare_mask - 1;
+            const int u = idx >> 2, k = idx & 3;
+            const int ml = ml0 + u * rstep;
+            const int m = m0 + ml;
+            int32_t a = 0;
+            for (int q = 0; q < p.splits; ++q)
+              a += static_cast<int32_t>(ld_dsmem_u32(mapa_shared(red_u32 + static_cast<uint32_t>((ml * 128 + nl + k) * 4), q)));
+            const RowConst<kW8A8> rk = row_const<kW8A8>(n + k, p);
+            reinterpret_cast<__half*>(p.Y)[static_cast<int64_t>(m) * p.N + n + k] =
+                epi_w8a8(a, __ldg(p.sx + m), rk);
           }
         }
       }
