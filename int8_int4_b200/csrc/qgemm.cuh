@@ -299,10 +299,23 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
                                                        const RowConst<KIND>& rc, const float* sxs) {
     uint32_t r[16];
     tmem_ld16(tacc + c * 16, r);
-    tmem_ld_wait();
     // transpose the warp's 32 channels x 16 tokens through shared memory
-    // ([16][32] box), then coalesced 16-byte stores along the channels
+    // ([16][32] box), then coalesced 16-byte stores along the channels.
+    // All shared-memory reads come before the first store into the box, and
+    // the 16 results are computed into registers first, so the elements are
+    // independent instruction streams.
+    __half h[16];
     if constexpr (KIND == kW8A8) {
+      float sxv[16];  // the chunk's 16 token scales, read while the TMEM load is in flight
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 f = reinterpret_cast<const float4*>(sxs + c * 16)[q];
+        sxv[4 * q + 0] = f.x;
+        sxv[4 * q + 1] = f.y;
+        sxv[4 * q + 2] = f.z;
+        sxv[4 * q + 3] = f.w;
+      }
+      tmem_ld_wait();
       // common path, straight-line over the chunk; elements flagged rare
       // are redone below from their accumulator, re-read from TMEM
       uint32_t rare_mask = 0;
@@ -310,8 +323,7 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           bool rare;
-          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-              w8a8_round_plain(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc.sw, rare);
+          h[i] = w8a8_round_plain(static_cast<int32_t>(r[i]), sxv[i], rc.sw, rare);
           rare_mask |= static_cast<uint32_t>(rare) << i;
         }
       } else {
@@ -319,11 +331,12 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
         for (int i = 0; i < 16; ++i) {
           bool rare;
           W8A8Val vv;
-          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-              w8a8_round(static_cast<int32_t>(r[i]), sxs[c * 16 + i], rc, vv, rare);
+          h[i] = w8a8_round(static_cast<int32_t>(r[i]), sxv[i], rc, vv, rare);
           rare_mask |= static_cast<uint32_t>(rare) << i;
         }
       }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = h[i];
       uint32_t any = __reduce_or_sync(0xffffffffu, rare_mask);
       while (any) {  // warp-uniform loop: the TMEM load is .sync.aligned
         const int i = __ffs(any) - 1;
@@ -340,14 +353,16 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
                          rc.has_bias, rc.has_steer, vv.yh, vv.yl);
         }
       }
-    } else {
+    } else if constexpr (KIND == kS32) {
+      tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if constexpr (KIND == kS32)
-          reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
-        else
-          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
-      }
+      for (int i = 0; i < 16; ++i) reinterpret_cast<uint32_t*>(sbuf)[i * 32 + lane] = r[i];
+    } else {
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) h[i] = epi_wo<KIND>(__uint_as_float(r[i]), rc);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = h[i];
     }
 }
 
