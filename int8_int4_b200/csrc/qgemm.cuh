@@ -485,17 +485,22 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
   const bool epi_warp = warp >= 4 && !(T::kDequant && warp >= 8);
 
+  // The producer and MMA roles run as whole converged warps: every lane waits,
+  // one lane issues (TMA by lane 0, MMA and commit by elect.sync), so the
+  // issue loops stay warp-uniform. Ring slots and phases advance
+  // incrementally (no division by the runtime ring depth in the loops).
   if (warp == 0) {
     // ------------------------------------------------ weight tile producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();  // weights are read once per m-tile
-      bool ok = true;
-      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
-        const int n0 = (tile % p.tiles_n) * kTileN;
-        if constexpr (T::kDequant) {
-          for (int i = 0; i < nu; ++i) {
-            const int s = issued_w % p.n_raw;
-            if (!(ok = mbar_wait(raw_empty + s, ((issued_w / p.n_raw) & 1) ^ 1, abort_flag, 1))) break;
+    const uint64_t pol = policy_evict_first();  // weights are read once per m-tile
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+      const int n0 = (tile % p.tiles_n) * kTileN;
+      if constexpr (T::kDequant) {
+        for (int i = 0; i < nu; ++i) {
+          if (!(ok = mbar_wait_warp(raw_empty + s, ph ^ 1, abort_flag, 1))) break;
+          if (lane == 0) {
             uint8_t* dst = raw + s * p.raw_stage;
             const int u = u_begin + i;
             if (i + kL2Ahead < nu) {  // keep the weight stream kL2Ahead units ahead in L2
@@ -510,84 +515,87 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
               tma_load_2d(&tmW, raw_full + s, dst, u * 128, n0, pol);        // 256 k as bytes
               tma_load_2d(&tmS, raw_full + s, dst + kATile, u * 8, n0, pol);  // 8 group scales
             }
-            ++issued_w;
           }
-        } else {
-          const uint64_t polx = policy_evict_last();
-          const int m0 = (tile / p.tiles_n) * p.BN;
-          for (int kb = 0; kb < nkb; ++kb) {
-            const int s = issued_w % p.n_a;
-            if (!(ok = mbar_wait(st_empty + s, ((issued_w / p.n_a) & 1) ^ 1, abort_flag, 2))) break;
+          ++issued_w;
+          if (++s == p.n_raw) { s = 0; ph ^= 1u; }
+        }
+      } else {
+        const uint64_t polx = policy_evict_last();
+        const int m0 = (tile / p.tiles_n) * p.BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2))) break;
+          if (lane == 0) {
             if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * 128, n0);
             mbar_arrive_expect_tx(st_full + s, kATile + p.x_stage);
             tma_load_2d(&tmW, st_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
             tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * 128, m0, polx);
-            ++issued_w;
           }
+          ++issued_w;
+          if (++s == p.n_a) { s = 0; ph ^= 1u; }
         }
       }
     }
   } else if (warp == 2 && T::kDequant) {
     // -------------------------------------------- activation tile producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_last();   // re-read by every weight tile
-      const int kx0 = u_begin * T::kKbPerUnit;
-      bool ok = true;
-      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
-        const int m0 = (tile / p.tiles_n) * p.BN;
-        for (int kb = 0; kb < nkb; ++kb) {
-          const int s = issued_x % p.n_a;
-          if (!(ok = mbar_wait(st_empty + s, ((issued_x / p.n_a) & 1) ^ 1, abort_flag, 3))) break;
+    const uint64_t pol = policy_evict_last();   // re-read by every weight tile
+    const int kx0 = u_begin * T::kKbPerUnit;
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+      const int m0 = (tile / p.tiles_n) * p.BN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 3))) break;
+        if (lane == 0) {
           mbar_arrive_expect_tx(st_full + s, p.x_stage);
           tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
-          ++issued_x;
         }
+        ++issued_x;
+        if (++s == p.n_a) { s = 0; ph ^= 1u; }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = T::kF16 ? idesc_f16_f32(p.BN) : idesc_s8_s32(p.BN);
-      int ka = 0, ti = 0;
-      bool ok = true;
-      for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
-        const int b = ti & 1;
-        if (!(ok = mbar_wait(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9))) break;
-        if (ti == 0) ARIA_STAMP(3);
+    const uint32_t idesc = T::kF16 ? idesc_f16_f32(p.BN) : idesc_s8_s32(p.BN);
+    int ti = 0, sa = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
+      const int b = ti & 1;
+      if (!(ok = mbar_wait_warp(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9))) break;
+      if (ti == 0 && lane == 0) ARIA_STAMP(3);
+      tc_fence_after();
+      const uint32_t dt = tmem_base + b * kAccCols;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!(ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4))) break;
+        if (kb == 0 && ti == 0 && lane == 0) ARIA_STAMP(4);
         tc_fence_after();
-        const uint32_t dt = tmem_base + b * kAccCols;
-        for (int kb = 0; kb < nkb; ++kb, ++ka) {
-          const int sa = ka % p.n_a, sx = sa;
-          ok = mbar_wait(st_full + sa, (ka / p.n_a) & 1, abort_flag, 4);
-          if (!ok) break;
-          if (ka == 0) ARIA_STAMP(4);
-          tc_fence_after();
-          const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
-          const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sx * p.x_stage));
+        const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
+        const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sa * p.x_stage));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
-            if constexpr (T::kF16)
-              umma_f16(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
-            else
-              umma_i8(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
-          }
-          umma_commit(st_empty + sa);  // releases both tiles of the stage
+        for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
+          if constexpr (T::kF16)
+            umma_f16_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+          else
+            umma_i8_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
         }
-        umma_commit(acc_full + b);  // also fires when nothing was issued
-        ARIA_STAMP(5);
+        umma_commit_elect(st_empty + sa);  // releases both tiles of the stage
+        if (++sa == p.n_a) { sa = 0; ph ^= 1u; }
       }
+      umma_commit_elect(acc_full + b);  // also fires when nothing was issued
+      if (lane == 0) ARIA_STAMP(5);
     }
   } else if (T::kDequant && warp >= 8) {
     // ------------------------------------------------------ dequantise
     if constexpr (T::kDequant) {
       const int t = threadIdx.x - 256;  // weight row within the tile
-      int ir = 0, ia = 0;
+      int s = 0, sa = 0;  // raw ring slot, stage ring slot
+      uint32_t rph = 0, aph = 0;
       bool ok = true;
       for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
-        for (int i = 0; i < nu && ok; ++i, ++ir) {
-          const int s = ir % p.n_raw;
-          if (!(ok = mbar_wait(raw_full + s, (ir / p.n_raw) & 1, abort_flag, 6))) break;
-          if (t == 0 && ir == 0) ARIA_STAMP(12);
+        for (int i = 0; i < nu && ok; ++i) {
+          if (!(ok = mbar_wait_fast(raw_full + s, rph, abort_flag, 6))) break;
+          if (t == 0 && tile == tile0 && i == 0) ARIA_STAMP(12);
           const uint8_t* src = raw + s * p.raw_stage;
           uint4 v[8];
 #pragma unroll
@@ -595,10 +603,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           uint4 sc = make_uint4(0, 0, 0, 0);
           if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
           mbar_arrive(raw_empty + s);
+          if (++s == p.n_raw) { s = 0; rph ^= 1u; }
 #pragma unroll
           for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
-            const int sa = ia % p.n_a;
-            if (!(ok = mbar_wait(st_empty + sa, ((ia / p.n_a) & 1) ^ 1, abort_flag, 7))) break;
+            if (!(ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7))) break;
             uint8_t* dst = abuf + sa * kATile;
             if constexpr (KIND == kQ8) {
               // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
@@ -630,7 +638,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             }
             fence_proxy_async_smem();
             mbar_arrive(st_full + sa);
-            ++ia;
+            if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
           }
         }
       }
@@ -838,7 +846,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
-  if (*abort_flag && lane == 0) {
+  const bool aborted = *abort_flag != 0;
+  if (aborted && lane == 0) {
     // drain copies still in flight into this CTA's shared memory
     // (q8/q4 stage barriers also wait for dequant arrivals, so only the raw
     // ring and W8A8 stages are drained here; X loads of q8/q4 stages were
@@ -851,10 +860,13 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     } else if (warp == 2 && issued_x > 0) {
       const uint64_t t0 = globaltimer();  // X loads of q8/q4: allow 100 us to land
       while (globaltimer() - t0 < 100000ull) __nanosleep(1000);
-    } else if (warp == 1) {
-      umma_commit(mma_drain);  // MMAs issued before the abort finish before TMEM is freed
-      mbar_wait_drain(mma_drain, 0);
     }
+  }
+  if (warp == 1 && __any_sync(0xffffffffu, aborted)) {
+    // MMAs issued before the abort finish before TMEM is freed; the commit
+    // comes from the lane that issued them (elect.sync, as in the issue loop)
+    umma_commit_elect(mma_drain);
+    mbar_wait_drain(mma_drain, 0);
   }
   tc_fence_before();
   __syncthreads();
