@@ -121,6 +121,7 @@ template <int KIND>
 struct RowConst {
   float sw = 0.0f, bias = 0.0f, alpha = 0.0f, v = 0.0f;  // all formats (W8A8: fp32 copies)
   float av_hi = 0.0f, av_lo = 0.0f;                      // W8A8: alpha*v = av_hi + av_lo exactly
+  float sw_up = 0.0f, sw_dn = 0.0f;                      // W8A8: sw * (1 +- 2^-21), rounded
   bool has_bias = false, has_steer = false;
 };
 
@@ -132,6 +133,8 @@ __device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) 
   c.has_steer = p.steer != nullptr;
   if constexpr (KIND == kW8A8) {
     c.sw = __ldg(p.sw + n);
+    c.sw_up = __fmul_rn(c.sw, 1.0f + 0x1p-21f);
+    c.sw_dn = __fmul_rn(c.sw, 1.0f - 0x1p-21f);
     if (c.has_bias) c.bias = __half2float(p.bias[n]);
     if (c.has_steer) {
       c.alpha = p.alpha;
@@ -237,8 +240,10 @@ __device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float
       half_gap = ldexpf(1.0f, e16 - (down_binade ? 12 : 11));
     }
     if (fabsf(d) == half_gap) {
+      // yh on the midpoint: yl != 0 decides the side; with yl == 0 the value
+      // is the midpoint itself and the conversion's tie-to-even stands
       const float yl_mag = yh < 0.0f ? -yl : yl;    // yl measured away from zero
-      if ((yl_mag > 0.0f) == (d > 0.0f)) {
+      if (yl_mag != 0.0f && (yl_mag > 0.0f) == (d > 0.0f)) {
         const uint32_t nb = d > 0.0f ? hb + 1u : hb - 1u;
         h = __ushort_as_half(static_cast<unsigned short>((__half_as_ushort(h) & 0x8000u) | nb));
       }
@@ -247,22 +252,26 @@ __device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float
   return h;
 }
 
-// No bias and no steering: y = fl(fl(acc) * fl(s_x*s_w)) is within 2 fp32 ulps
-// of the exact product E (acc is exact in fp32 below 2^22), so RN16(y) ==
-// RN16(E) unless y's 13 bits below fp16 precision are within 3 of the
-// midpoint pattern 0x1000, or y is outside the fp16 normal range; those
-// (about 0.1 % of elements) are flagged `rare` for the exact path.
-__device__ __forceinline__ __half w8a8_round_plain(int32_t acc, float sx, float sw, bool& rare) {
-  const float a = __fsub_rn(__int_as_float(acc + 0x4B400000), 12582912.0f);  // exact if |acc| < 2^22
-  const float y = __fmul_rn(a, __fmul_rn(sx, sw));
-  const uint32_t yb = __float_as_uint(y) & 0x7FFFFFFFu;
-  const uint32_t low = yb & 0x1FFFu;
-  rare = (low - 0x0FFDu) <= 6u                              // |low - 0x1000| <= 3
-         || (yb - 0x38800000u) >= (0x477FF000u - 0x38800000u) // |y| < 2^-14 or |y| >= 65504 - 16
-         || static_cast<uint32_t>(acc + (1 << 22) - 1) >= static_cast<uint32_t>((1 << 23) - 1);
-  rare = rare && y != 0.0f;  // an exact zero rounds to itself
-  return __float2half_rn(y);
+// No bias and no steering. With t = fl(fl(acc) * s_x), the two products
+// y_up = fl(t * fl(s_w (1 + 2^-21))) and y_dn = fl(t * fl(s_w (1 - 2^-21)))
+// bracket the reference value E = fl64(fl64(acc * s_x) * s_w): the four fp32
+// roundings on each side (acc, t, the scaled s_w, the product) move a value
+// by at most 4 * 2^-24 relative, less than the 2^-21 margin. Rounding to
+// fp16 is monotonic, so if y_up and y_dn round to the same fp16 value, E
+// does too. One packed conversion rounds both; the halves differ for about
+// 0.1 % of elements (E near an fp16 rounding midpoint), which the caller
+// recomputes with the fp64 sequence. No range check on acc is needed: the
+// int-to-float conversion is one of the four roundings.
+__device__ __forceinline__ uint32_t w8a8_plain_pair(int32_t acc, float sx, float sw_up, float sw_dn) {
+  const float t = __fmul_rn(__int2float_rn(acc), sx);
+  const float yu = __fmul_rn(t, sw_up);
+  const float yd = __fmul_rn(t, sw_dn);
+  uint32_t pk;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(pk) : "f"(yu), "f"(yd));
+  return pk;  // low half RN16(y_dn), high half RN16(y_up)
 }
+
+__device__ __forceinline__ bool pair_split(uint32_t pk) { return (pk >> 16) != (pk & 0xFFFFu); }
 
 __device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst<kW8A8>& c) {
   W8A8Val v;
@@ -316,15 +325,15 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
         sxv[4 * q + 3] = f.w;
       }
       tmem_ld_wait();
-      // common path, straight-line over the chunk; elements flagged rare
-      // are redone below from their accumulator, re-read from TMEM
+      // common path, straight-line over the chunk; each lane then redoes its
+      // own flagged elements (registers selected by index, no TMEM re-read)
       uint32_t rare_mask = 0;
       if (!rc.has_bias && !rc.has_steer) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          bool rare;
-          h[i] = w8a8_round_plain(static_cast<int32_t>(r[i]), sxv[i], rc.sw, rare);
-          rare_mask |= static_cast<uint32_t>(rare) << i;
+          const uint32_t pk = w8a8_plain_pair(static_cast<int32_t>(r[i]), sxv[i], rc.sw_up, rc.sw_dn);
+          h[i] = __ushort_as_half(static_cast<unsigned short>(pk & 0xFFFFu));
+          rare_mask |= static_cast<uint32_t>(pair_split(pk)) << i;
         }
       } else {
 #pragma unroll
@@ -337,21 +346,29 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = h[i];
-      uint32_t any = __reduce_or_sync(0xffffffffu, rare_mask);
-      while (any) {  // warp-uniform loop: the TMEM load is .sync.aligned
-        const int i = __ffs(any) - 1;
-        any &= any - 1;
-        const uint32_t a1 = tmem_ld1(tacc + c * 16 + i);
-        tmem_ld_wait();
-        if (rare_mask & (1u << i)) {
-          const float sxi = sxs[c * 16 + i];
+      while (rare_mask) {
+        const int i = __ffs(rare_mask) - 1;
+        rare_mask &= rare_mask - 1;
+        uint32_t a1 = r[0];
+        float sxi = sxv[0];
+#pragma unroll
+        for (int k = 1; k < 16; ++k) {
+          if (k == i) {
+            a1 = r[k];
+            sxi = sxv[k];
+          }
+        }
+        __half hv;
+        if (!rc.has_bias && !rc.has_steer) {
+          hv = epi_w8a8_fp64(static_cast<int32_t>(a1), sxi, rc.sw, 0.0f, 0.0f, 0.0f, false, false);
+        } else {
           bool rare;
           W8A8Val vv;
           const __half h0 = w8a8_round(static_cast<int32_t>(a1), sxi, rc, vv, rare);
-          reinterpret_cast<__half*>(sbuf)[i * 32 + lane] =
-              w8a8_fixup(h0, static_cast<int32_t>(a1), sxi, rc.sw, rc.bias, rc.alpha, rc.v,
-                         rc.has_bias, rc.has_steer, vv.yh, vv.yl);
+          hv = w8a8_fixup(h0, static_cast<int32_t>(a1), sxi, rc.sw, rc.bias, rc.alpha, rc.v,
+                          rc.has_bias, rc.has_steer, vv.yh, vv.yl);
         }
+        reinterpret_cast<__half*>(sbuf)[i * 32 + lane] = hv;
       }
     } else if constexpr (KIND == kS32) {
       tmem_ld_wait();
@@ -806,7 +823,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
               for (int k = 0; k < 4; ++k) {
                 bool rare;
                 if (!rc[k].has_bias && !rc[k].has_steer) {
-                  h[k] = w8a8_round_plain(static_cast<int32_t>(a4[k]), sxm, rc[k].sw, rare);
+                  const uint32_t pk = w8a8_plain_pair(static_cast<int32_t>(a4[k]), sxm, rc[k].sw_up, rc[k].sw_dn);
+                  h[k] = __ushort_as_half(static_cast<unsigned short>(pk & 0xFFFFu));
+                  rare = pair_split(pk);
                 } else {
                   W8A8Val vv;
                   h[k] = w8a8_round(static_cast<int32_t>(a4[k]), sxm, rc[k], vv, rare);

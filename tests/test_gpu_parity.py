@@ -135,6 +135,40 @@ def test_w8a8_within_one_ulp(M, N, K, bias, steer):
                       None if b is None else b.numpy(), None if v is None else v.numpy(), alpha)
     d = ulp_dist(Y.cpu().numpy().view(np.uint16), ref)
     assert d.max() <= 1, d.max()
+    assert (d == 0).all(), (d != 0).sum()  # the epilogue rounds exactly
+
+
+@pytest.mark.parametrize("M,N,K", [(96, 256, 512),      # 2 tiles: split-K cluster reduction
+                                   (4096, 1280, 256)])  # 160 tiles: persistent epilogue
+@pytest.mark.parametrize("bias,steer", [(False, False), (True, False), (True, True)])
+def test_w8a8_exact_fp16_ties_round_to_even(M, N, K, bias, steer):
+    """s_x = 2^-5 and s_w = 2^-11 make acc * s_x * s_w = acc * 2^-16 exact in
+    binary, so every odd |acc| in [2^11, 2^12) (and many others) lands exactly
+    on an fp16 rounding midpoint; the result must be the tie-to-even value."""
+    rng = np.random.default_rng(11)
+    xc = rng.integers(-127, 128, (M, K)); xc[:, 0] = rng.choice([-127, 127], M)
+    wc = rng.integers(-127, 128, (N, K)); wc[:, 0] = rng.choice([-127, 127], N)
+    X = torch.from_numpy((xc * 2.0 ** -5).astype(np.float16))     # row absmax 127 * 2^-5
+    W = torch.from_numpy((wc * 2.0 ** -11).astype(np.float16))    # row absmax 127 * 2^-11
+    Wq, sw = aq.qpack("q8", W.cuda())
+    Xq, sx = aq.act_quant(X.cuda())
+    assert (sx == 2.0 ** -5).all() and (sw == 2.0 ** -11).all()
+    key = "gpu/w8a8ties"
+    b = synthetic.bias(key, N) if bias else None
+    v = synthetic.steer_vec(key, N) if steer else None
+    alpha = 0.3 if steer else 0.0
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx, bias=None if b is None else b.cuda(),
+                 steer_vec=None if v is None else v.cuda(), alpha=alpha)
+    rows = sample_rows(M, 48) if M > 256 else None
+    ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(),
+                      None if b is None else b.numpy(), None if v is None else v.numpy(), alpha, rows=rows)
+    if not bias:
+        acc = (xc if rows is None else xc[rows]) @ wc.T
+        assert ((np.abs(acc) >= 2 ** 11) & (np.abs(acc) < 2 ** 12) & (acc % 2 == 1)).sum() > 100
+    got = Y.cpu().numpy().view(np.uint16)
+    if rows is not None:
+        got = got[rows]
+    assert np.array_equal(got, ref), (got != ref).sum()
 
 
 def test_w8a8_large_accumulators_take_exact_path():
