@@ -500,7 +500,6 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 
   int issued_w = 0, issued_x = 0;  // kept for the teardown drain
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
-  const bool epi_warp = warp >= 4 && !(T::kDequant && warp >= 8);
 
   // The producer and MMA roles run as whole converged warps: every lane waits,
   // one lane issues (TMA by lane 0, MMA and commit by elect.sync), so the
@@ -619,6 +618,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(src + sw128(t, c));
           uint4 sc = make_uint4(0, 0, 0, 0);
           if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
+          // The slot's next writer is a TMA load (async proxy): order this
+          // thread's generic-proxy reads of it before that write. Without
+          // the proxy fence the release of the arrive alone let a refill land
+          // before the reads of v[4..7] completed (measured: wrong second A
+          // tile of a unit in about 1 of 3 launches at M = 4096).
+          fence_proxy_async_smem();
           mbar_arrive(raw_empty + s);
           if (++s == p.n_raw) { s = 0; rph ^= 1u; }
 #pragma unroll
@@ -736,28 +741,27 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         }
         if (te == 0) ARIA_STAMP(7);
       }
-    } else {
-      // split-K: one tile per CTA; wait for its partial accumulator
-      bool ok = mbar_wait(acc_full, 0, abort_flag, 8);
-      epi_ok = __all_sync(0xffffffffu, ok);
     }
   }
 
   // ------------------------------------------- split-K: cluster reduction
-  // Each CTA first writes its partial tile to its own shared memory,
-  // red[m_local][128] (32-bit words, overlaying the now idle stage rings).
-  // After a cluster barrier, rank r reduces token rows [BN*r/S, BN*(r+1)/S),
-  // summing the S partials in rank order (deterministic) with
-  // distributed-shared-memory loads, four rows in flight per thread.
+  // One tile per CTA. Once its partial accumulator is complete every role
+  // has finished, so all 12 warps take part: each writes a third of its
+  // TMEM lane group's columns to red[m_local][128] (32-bit words, overlaying
+  // the idle stage rings). After a cluster barrier, rank r reduces token rows
+  // [BN*r/S, BN*(r+1)/S): each thread keeps one group of 4 channels, issues
+  // the distributed-shared-memory loads of all S partials for two rows at
+  // once, then sums them in rank order (deterministic) and applies the
+  // epilogue.
   if (split) {
-    if (epi_warp) {
-      const int e = warp - 4;
-      const int t = (warp & 3) * 32 + lane;
-      const int cgrp = e >> 2, cstep = T::kEpiWarps >> 2;
-      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    epi_ok = mbar_wait_warp(acc_full, 0, abort_flag, 8);
+    const int lg = warp & 3, wg = warp >> 2;  // TMEM lane group; third of the columns
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem);
+    {
+      const int t = lg * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
       tc_fence_after();
-      uint32_t* red = reinterpret_cast<uint32_t*>(smem);
-      for (int c = cgrp; c < p.BN / 16; c += cstep) {
+      for (int c = wg; c < p.BN / 16; c += 3) {
         uint32_t r[16];
         tmem_ld16(tmem_base + lane_off + c * 16, r);
         tmem_ld_wait();
@@ -768,47 +772,49 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     __syncwarp();
     cluster_sync();
     ARIA_STAMP(8);
-    if (epi_warp) {
-      const int te = threadIdx.x - 128;
-      const int rstep = T::kEpiWarps;  // rows advanced per pass (32 threads per row)
+    {
+      constexpr int kWarps = KindTraits<KIND>::kThreads / 32;
+      constexpr int kRows = 2;       // rows in flight per thread
+      constexpr int kMaxSplits = 8;
       const int n0 = (tile0 % p.tiles_n) * kTileN;
       const int m0 = (tile0 / p.tiles_n) * p.BN;
       const int mb = p.BN * rank / p.splits, me = p.BN * (rank + 1) / p.splits;
-      const int nl = (te & 31) * 4;
+      const int nl = lane * 4;
       const int n = n0 + nl;
       RowConst<KIND> rc[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) rc[j] = row_const<KIND>(n + j, p);
       const uint32_t red_u32 = smem_u32(smem);
-      constexpr int kRows = 4;
-      for (int ml0 = mb + (te >> 5); ml0 < me; ml0 += kRows * rstep) {
+      for (int ml0 = mb + warp; ml0 < me; ml0 += kRows * kWarps) {
+        uint4 v[kMaxSplits][kRows];
+#pragma unroll
+        for (int q = 0; q < kMaxSplits; ++q) {
+#pragma unroll
+          for (int u = 0; u < kRows; ++u) {
+            const int ml = ml0 + u * kWarps;
+            v[q][u] = make_uint4(0u, 0u, 0u, 0u);
+            if (q < p.splits && ml < me)
+              v[q][u] = ld_dsmem_v4(mapa_shared(red_u32 + static_cast<uint32_t>((ml * 128 + nl) * 4), q));
+          }
+        }
         uint4 acc[kRows];
 #pragma unroll
-        for (int u = 0; u < kRows; ++u) acc[u] = make_uint4(0, 0, 0, 0);
-        for (int q = 0; q < p.splits; ++q) {
-          uint4 v[kRows];
+        for (int u = 0; u < kRows; ++u) {
+          acc[u] = v[0][u];
 #pragma unroll
-          for (int u = 0; u < kRows; ++u) {
-            const int ml = ml0 + u * rstep;
-            if (ml < me)
-              v[u] = ld_dsmem_v4(mapa_shared(red_u32 + static_cast<uint32_t>((ml * 128 + nl) * 4), q));
-          }
-#pragma unroll
-          for (int u = 0; u < kRows; ++u) {
-            if (q == 0) {
-              acc[u] = v[u];
-            } else {
-              acc[u].x = reduce_add<KIND>(acc[u].x, v[u].x);
-              acc[u].y = reduce_add<KIND>(acc[u].y, v[u].y);
-              acc[u].z = reduce_add<KIND>(acc[u].z, v[u].z);
-              acc[u].w = reduce_add<KIND>(acc[u].w, v[u].w);
+          for (int q = 1; q < kMaxSplits; ++q) {
+            if (q < p.splits) {
+              acc[u].x = reduce_add<KIND>(acc[u].x, v[q][u].x);
+              acc[u].y = reduce_add<KIND>(acc[u].y, v[q][u].y);
+              acc[u].z = reduce_add<KIND>(acc[u].z, v[q][u].z);
+              acc[u].w = reduce_add<KIND>(acc[u].w, v[q][u].w);
             }
           }
         }
         uint32_t rare_mask = 0;  // W8A8: elements to redo exactly (bit 4u+k)
 #pragma unroll
         for (int u = 0; u < kRows; ++u) {
-          const int ml = ml0 + u * rstep;
+          const int ml = ml0 + u * kWarps;
           const int m = m0 + ml;
           if (ml >= me || m >= p.M || n >= p.N) continue;  // N % 16 == 0: 4 columns in range
           const int64_t o = static_cast<int64_t>(m) * p.N + n;
@@ -846,7 +852,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             const int idx = __ffs(rare_mask) - 1;
             rare_mask &= rare_mask - 1;
             const int u = idx >> 2, k = idx & 3;
-            const int ml = ml0 + u * rstep;
+            const int ml = ml0 + u * kWarps;
             const int m = m0 + ml;
             int32_t a = 0;
             for (int q = 0; q < p.splits; ++q)

@@ -296,6 +296,25 @@ def test_alpha_zero_is_bit_identical(fmt):
 
 
 @pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
+def test_repeated_launches_bit_identical(fmt):
+    """Persistent multi-tile launches (M = 4096: several tiles per CTA, rings
+    wrapping many times) give bit-identical results run after run; a
+    cross-proxy ordering race on the raw-weight ring showed up here as a few
+    wrong weight rows in about one launch in three."""
+    M, N, K = 4096, 6144, 1536
+    key = f"gpu/repeat/{fmt}"
+    W = synthetic.weight(f"{key}/W", N, K).cuda()
+    X = synthetic.activation(key, M, K).cuda()
+    Wq, sc = aq.qpack("q8" if fmt == "w8a8" else fmt, W)
+    sx = None
+    if fmt == "w8a8":
+        X, sx = aq.act_quant(X)
+    outs = [aq.qgemm(fmt, X, Wq, sc, sx=sx) for _ in range(12)]
+    for i, Y in enumerate(outs[1:], 1):
+        assert torch.equal(Y, outs[0]), (i, int((Y != outs[0]).sum()))
+
+
+@pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
 def test_deterministic_split_k(fmt):
     M, N, K = 1, 1024, 4096                        # few tiles: split-K across a cluster
     W = synthetic.weight(f"gpu/det/{fmt}/W", N, K)
