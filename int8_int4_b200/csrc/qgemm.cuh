@@ -445,7 +445,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   uint64_t* acc_full = st_empty + p.n_a;  // [2]
   uint64_t* acc_empty = acc_full + 2;     // [2]
   uint64_t* mma_drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  // single use: the CTA's last tile is complete. The dequant warps, which
+  // leave their role early to help with that tile, wait on it rather than
+  // on acc_full, whose parity could alias when they run several tiles ahead
+  // of the MMA (short K, many tiles per CTA)
+  uint64_t* acc_last = mma_drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_last + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
@@ -463,6 +468,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       mbar_init(acc_empty + i, T::kEpiWarps);
     }
     mbar_init(mma_drain, 1);
+    mbar_init(acc_last, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -599,6 +605,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         if (++sa == p.n_a) { sa = 0; ph ^= 1u; }
       }
       umma_commit_elect(acc_full + b);  // also fires when nothing was issued
+      if (tile + tstep >= p.tiles) umma_commit_elect(acc_last);
       if (lane == 0) ARIA_STAMP(5);
     }
   } else if (T::kDequant && warp >= 8) {
@@ -673,7 +680,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         const int n0 = (tile % p.tiles_n) * kTileN;
         const int m0 = (tile / p.tiles_n) * p.BN;
         const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
-        bool ok2 = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 10);
+        bool ok2 = mbar_wait(acc_last, 0, abort_flag, 10);
         ok2 = __all_sync(0xffffffffu, ok2);
         if (ok2) {
           tc_fence_after();

@@ -295,6 +295,25 @@ def test_alpha_zero_is_bit_identical(fmt):
     assert diff.abs().max().item() < 2e-3          # y + alpha*v, up to fp16 rounding
 
 
+@pytest.mark.parametrize("fmt,K", [("q8", 128), ("q4", 256), ("w8a8", 128), ("w8a8", 256)])
+def test_small_k_many_tiles(fmt, K):
+    """Short K with hundreds of output tiles: the producer and dequant warps
+    finish their rings several tiles ahead of the MMA and then join the last
+    tile's epilogue; they must wait for that tile, not an earlier one that
+    shares its accumulator buffer."""
+    M, N = 4096, 6144
+    rows = sample_rows(M, 16)
+    key = f"gpu/smallk/{fmt}/{K}"
+    if fmt == "w8a8":
+        X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, key)
+        Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx)
+        ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(), rows=rows)
+        assert np.array_equal(Y.cpu().numpy().view(np.uint16)[rows], ref)
+    else:
+        y, ref = _wo(fmt, M, N, K, key, rows=rows)
+        check_wo(y, ref)
+
+
 @pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
 def test_repeated_launches_bit_identical(fmt):
     """Persistent multi-tile launches (M = 4096: several tiles per CTA, rings
