@@ -124,6 +124,16 @@ aria_status aria_act_quant(const void *X, int64_t M, int64_t K, int8_t *Xq, floa
  * Shape rules: M >= 1; N >= 16, N % 16 == 0; K >= 16, K % 16 == 0;
  *   Q4 additionally K % 256 == 0; group as in aria_qpack_size.
  * Deterministic: the same inputs give the same bytes on every call.
+ * Stream order: the kernel is launched with programmatic dependent launch,
+ *   so it may start while the preceding kernel in `stream` finishes. X, sx,
+ *   bias, steer_vec and Y are touched only after that kernel has completed;
+ *   the first weight tiles (Wq, and the Q4 scales) are loaded before. Wq and
+ *   scales must therefore be complete before the preceding kernel in the
+ *   stream starts, or be written by a kernel that does not allow an early
+ *   start of its successor (no griddepcontrol.launch_dependents /
+ *   cudaTriggerProgrammaticLaunchCompletion before its last write).
+ *   aria_qpack's kernels never allow it, so pack-then-GEMM on one stream is
+ *   safe.
  */
 aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
                        const void *X, const float *sx, const void *Wq, const void *scales,

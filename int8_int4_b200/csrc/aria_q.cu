@@ -348,7 +348,8 @@ ARIA_API aria_status aria_qpack(aria_format fmt, int group, const void* W, int64
     cfg.gridDim = dim3(static_cast<unsigned>(N));
     cfg.blockDim = dim3(aria::kRowThreads);
     e = cudaLaunchKernelEx(&cfg, aria::row_quant_i8_kernel, static_cast<const __half*>(W),
-                           static_cast<int>(K), static_cast<int8_t*>(Wq), static_cast<float*>(scales));
+                           static_cast<int>(K), static_cast<int8_t*>(Wq), static_cast<float*>(scales),
+                           false);
   }
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   return ARIA_OK;
@@ -369,7 +370,7 @@ ARIA_API aria_status aria_act_quant(const void* X, int64_t M, int64_t K, int8_t*
   cfg.blockDim = dim3(aria::kRowThreads);
   set_pdl(cfg, attr);
   cudaError_t e = cudaLaunchKernelEx(&cfg, aria::row_quant_i8_kernel, static_cast<const __half*>(X),
-                                     static_cast<int>(K), Xq, sx);
+                                     static_cast<int>(K), Xq, sx, true);
   if (e != cudaSuccess) return cuda_fail(e, "act_quant launch");
   return ARIA_OK;
 }

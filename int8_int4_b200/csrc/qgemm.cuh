@@ -485,26 +485,57 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Weights start moving into L2 while the preceding kernel drains: an L2
-  // prefetch is safe even if that kernel were still writing them (L2 is
-  // coherent), and the shared-memory loads below only start after the wait.
-  if (warp == 0 && lane == 0 && tile0 < p.tiles) {
+  // Programmatic dependent launch: this CTA may start while the preceding
+  // kernel in the stream drains. Packed weights and their scales are inputs
+  // that no kernel of this library writes while a following GEMM can already
+  // run (the pack kernels do not allow an early start; the header states the
+  // rule for callers), so the first ring of weight tiles is loaded before
+  // the wait: the raw units of the first tile (q8/q4) or the weight half of
+  // its first stages (W8A8, whose activation half follows after the wait on
+  // the same barrier). Activations, their scales and the output wait for
+  // the preceding kernel to complete.
+  int issued_w = 0, issued_x = 0;  // kept for the teardown drain
+  int pre = 0;                     // raw units / stages of the first tile issued before the wait
+  if (warp == 0 && tile0 < p.tiles) {
     const int n0 = (tile0 % p.tiles_n) * kTileN;
-    const int npf = nu < kL2Ahead ? nu : kL2Ahead;
-    for (int i = 0; i < npf; ++i) {
-      tma_prefetch_2d(&tmW, (u_begin + i) * 128, n0);
-      if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
+    const uint64_t pol = policy_evict_first();
+    if constexpr (T::kDequant) {
+      pre = nu < p.n_raw ? nu : p.n_raw;
+      if (lane == 0) {
+        for (int i = 0; i < pre; ++i) {
+          const int u = u_begin + i;
+          uint8_t* dst = raw + i * p.raw_stage;
+          if constexpr (KIND == kQ8) {
+            mbar_arrive_expect_tx(raw_full + i, kATile);
+            tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
+          } else {
+            mbar_arrive_expect_tx(raw_full + i, kATile + kQ4ScaleTile);
+            tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
+            tma_load_2d(&tmS, raw_full + i, dst + kATile, u * 8, n0, pol);
+          }
+        }
+      }
+    } else {
+      pre = nkb < p.n_a ? nkb : p.n_a;
+      if (lane == 0) {
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(st_full + i, kATile + p.x_stage);
+          tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * 128, n0, pol);
+        }
+      }
+    }
+    issued_w = pre;
+    if (lane == 0) {  // and the next units into L2
+      for (int i = pre; i < nu && i < pre + kL2Ahead; ++i) {
+        tma_prefetch_2d(&tmW, (u_begin + i) * 128, n0);
+        if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
+      }
     }
   }
-  // Inputs may come from the preceding kernel in the stream (programmatic
-  // dependent launch): everything above overlapped its tail; nothing below
-  // reads or writes global memory before it has completed.
   if (threadIdx.x == 0) ARIA_STAMP(1);
   pdl_wait();
   pdl_launch_dependents();
   if (threadIdx.x == 0) ARIA_STAMP(2);
-
-  int issued_w = 0, issued_x = 0;  // kept for the teardown drain
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
 
   // The producer and MMA roles run as whole converged warps: every lane waits,
@@ -521,6 +552,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       const int n0 = (tile % p.tiles_n) * kTileN;
       if constexpr (T::kDequant) {
         for (int i = 0; i < nu; ++i) {
+          if (tile == tile0 && i < pre) {  // issued before the dependency wait
+            if (++s == p.n_raw) { s = 0; ph ^= 1u; }
+            continue;
+          }
           if (!(ok = mbar_wait_warp(raw_empty + s, ph ^ 1, abort_flag, 1))) break;
           if (lane == 0) {
             uint8_t* dst = raw + s * p.raw_stage;
@@ -545,6 +580,14 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         const uint64_t polx = policy_evict_last();
         const int m0 = (tile / p.tiles_n) * p.BN;
         for (int kb = 0; kb < nkb; ++kb) {
+          if (tile == tile0 && kb < pre) {
+            // the weight half went out before the dependency wait (the barrier
+            // already expects both halves): add the activation half
+            if (lane == 0)
+              tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * 128, m0, polx);
+            if (++s == p.n_a) { s = 0; ph ^= 1u; }
+            continue;
+          }
           if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2))) break;
           if (lane == 0) {
             if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * 128, n0);

@@ -49,12 +49,17 @@ __device__ __forceinline__ uint2 quant8_i8(const uint4& v, float s, bool zero) {
 // One CTA per row: s[r] = absmax / 127, q = clamp(rhe(x / s), -127, 127).
 // Row r of X starts 16-byte aligned (K % 8 == 0); the first kRowCached
 // chunks of each thread stay in registers between the two passes.
+// `early_dependents`: let the next kernel in the stream start its set-up
+// now (activation quantisation). Weight packing passes false: a GEMM reads
+// packed weights before it waits for the preceding kernel, so it must not
+// start before the pack has finished.
 __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half* __restrict__ X,
                                                                    int K, int8_t* __restrict__ Q,
-                                                                   float* __restrict__ S) {
+                                                                   float* __restrict__ S,
+                                                                   bool early_dependents) {
   __shared__ float warp_max[kRowThreads / 32];
   pdl_wait();  // X may be written by the preceding kernel
-  pdl_launch_dependents();
+  if (early_dependents) pdl_launch_dependents();
   const int64_t r = blockIdx.x;
   const int nchunk = K >> 3;
   const uint4* xr = reinterpret_cast<const uint4*>(X + r * static_cast<int64_t>(K));
@@ -97,13 +102,13 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half*
 // consecutive lanes form a group of 32 and share its absmax by shuffles.
 // s16 = fp16_rn(absmax / 7); code = clamp(rhe(w / float(s16)), -7, 7) + 8,
 // even k in the low nibble. Loop bounds are warp-uniform so every lane
-// takes part in the shuffles.
+// takes part in the shuffles. No early start of the next kernel: a GEMM
+// reads packed weights before it waits for the preceding kernel.
 __global__ void __launch_bounds__(256) pack_q4_kernel(const __half* __restrict__ W,
                                                       int64_t nchunk,
                                                       uint32_t* __restrict__ P,
                                                       __half* __restrict__ S) {
   pdl_wait();
-  pdl_launch_dependents();
   const uint4* w4 = reinterpret_cast<const uint4*>(W);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x; base < nchunk;
