@@ -43,7 +43,9 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # ARIA_ORACLE_LIB: a separately compiled oracle library, used by the
+            # mutation tests to run the pins against a copy with a planted mistake
+            lib = ctypes.CDLL(os.environ.get("ARIA_ORACLE_LIB") or build())
             P, I64, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
             sigs = {
                 "orc_half_to_double": ([ctypes.c_uint16], ctypes.c_double),

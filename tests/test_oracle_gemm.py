@@ -41,6 +41,14 @@ def test_gemm_s32_extremes_and_overflow():
     Kbig = (2 ** 31) // (127 * 127) + 1
     with pytest.raises(OverflowError):
         oracle.gemm_s32(np.full((1, Kbig), 127, np.int8), np.full((1, Kbig), 127, np.int8))
+    # below INT32_MIN as well (sum of -127 * 127 terms)
+    Kneg = (2 ** 31) // (127 * 127) + 2
+    with pytest.raises(OverflowError):
+        oracle.gemm_s32(np.full((1, Kneg), 127, np.int8), np.full((1, Kneg), -127, np.int8))
+    # and just inside the range: no error, exact value
+    Kok = (2 ** 31 - 1) // (127 * 127)
+    C = oracle.gemm_s32(np.full((1, Kok), -127, np.int8), np.full((1, Kok), 127, np.int8))
+    assert C[0, 0] == -127 * 127 * Kok
 
 
 def _half_rne_exact(x: Fraction) -> int:

@@ -81,6 +81,25 @@ def test_q8_error_bound_and_extremes(N, K, std):
     assert np.all(np.abs(s.astype(np.float64) - a / 127) <= a / 127 * 2.0 ** -24)
 
 
+def test_q8_codes_match_ieee_fp32_rule():
+    """Brute force against an independent statement of the rule with numpy's
+    IEEE fp32 arithmetic: s = fp32(absmax / 127), q = rint(fp32(x / s)) (half
+    to even), over a million fp16 values at many scales. Codes near .5 tell a
+    correctly rounded quotient from, e.g., x * (1 / s)."""
+    rng = np.random.default_rng(0)
+    R, K = 4000, 256
+    X16 = (rng.standard_normal((R, K)) * rng.uniform(0.01, 10, (R, 1))).astype(np.float16)
+    X = X16.astype(np.float32)
+    a = np.abs(X).max(axis=1, keepdims=True)
+    s = (a / np.float32(127)).astype(np.float32)
+    q = np.clip(np.rint((X / s).astype(np.float32)), -127, 127).astype(np.int8)
+    Wq, sw = oracle.pack_q8(X16)
+    assert np.array_equal(sw, s[:, 0])
+    assert np.array_equal(Wq, q)
+    Xq, sx = oracle.act_quant(X16)
+    assert np.array_equal(sx, s[:, 0]) and np.array_equal(Xq, q)
+
+
 def test_q8_zero_and_identity():
     Z = np.zeros((16, 32), np.float16)
     Wq, s = oracle.pack_q8(Z)
