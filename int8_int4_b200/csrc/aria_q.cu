@@ -122,12 +122,41 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
 #if defined(ARIA_MAX_BN)
   max_bn = ARIA_MAX_BN;  // tuning builds only
 #endif
-  int mt = static_cast<int>((M + max_bn - 1) / max_bn);
-  int bn = static_cast<int>((M + mt - 1) / mt);
-  bn = (bn + 15) / 16 * 16;
-  mt = static_cast<int>((M + bn - 1) / bn);
-  p.BN = bn;
+  auto tile_for = [&](int mt_try, int* bn_out) {  // token tile for mt_try token tiles
+    int b = static_cast<int>((M + mt_try - 1) / mt_try);
+    b = (b + 15) / 16 * 16;
+    *bn_out = b;
+    return static_cast<int>((M + b - 1) / b);
+  };
+  int bn = 0;
+  int mt = tile_for(static_cast<int>((M + max_bn - 1) / max_bn), &bn);
   const int nt = static_cast<int>((N + kTileN - 1) / kTileN);
+  // q8/q4 with a few hundred tokens: the dequant work per K block is the
+  // same for any token tile, and a split-K launch costs several us of
+  // cluster reduction. Measured at M = 432 (d = 1536 linears): prefer the
+  // token tile that fills the most SMs (at least two thirds) without split-K;
+  // otherwise one tile narrower than the widest when K is short (fewer
+  // ranks to reduce), the widest when K is long (less K per rank).
+  bool dq_policy = (kind == kQ8 || kind == kQ4) && M >= 128 && M <= 512;
+#if defined(ARIA_MAX_BN)
+  dq_policy = false;  // tuning builds pin the tile
+#endif
+  if (dq_policy) {
+    const int mt0 = mt;
+    int best_mt = 0, best_tiles = 0;
+    for (int m_try = mt0; m_try <= mt0 + 2; ++m_try) {
+      int b = 0;
+      const int m_eff = tile_for(m_try, &b);
+      const int64_t t = static_cast<int64_t>(nt) * m_eff;
+      if (t <= di.sms && 3 * t >= 2 * static_cast<int64_t>(di.sms) && t > best_tiles) {
+        best_tiles = static_cast<int>(t);
+        best_mt = m_try;
+      }
+    }
+    if (best_mt == 0) best_mt = K <= 2048 ? mt0 + 1 : mt0;
+    mt = tile_for(best_mt, &bn);
+  }
+  p.BN = bn;
   const int64_t tiles = static_cast<int64_t>(nt) * mt;
   if (tiles > (int64_t{1} << 30)) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
   p.tiles_n = nt;
