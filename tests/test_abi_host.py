@@ -87,3 +87,47 @@ def test_no_cpu_path():
     import torch
     with pytest.raises(ValueError):
         aq.act_quant(torch.zeros(4, 16, dtype=torch.float16))
+
+
+OK_PTR = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("fmt,group,M,N,K,status", [
+    (1, 0, 0, 16, 16, 1),            # M < 1
+    (1, 0, 4, 0, 16, 1),             # N < 1
+    (1, 0, 4, 16, -16, 1),           # K < 1
+    (1, 0, 2 ** 31, 16, 16, 1),      # a dimension >= 2^31
+    (1, 0, 4, 8, 16, 2),             # N < 16
+    (1, 0, 4, 24, 16, 2),            # N % 16
+    (1, 0, 4, 16, 8, 2),             # K < 16
+    (1, 0, 4, 16, 40, 2),            # K % 16
+    (2, 32, 4, 16, 128, 2),          # q4 GEMM: K % 256
+    (3, 0, 4, 16, 24, 2),            # W8A8: K % 16
+    (1, 32, 4, 16, 16, 2),           # q8 takes group 0
+    (2, 0, 4, 16, 256, 2),           # q4 takes group 32
+])
+def test_qgemm_shape_rules(lib, fmt, group, M, N, K, status):
+    sx = OK_PTR if fmt == 3 else None
+    assert lib.aria_qgemm(fmt, group, M, N, K, OK_PTR, sx, OK_PTR, OK_PTR, None, None, 0.0, OK_PTR,
+                          None) == status
+    assert lib.aria_last_error_message()
+
+
+@pytest.mark.parametrize("M,N,K,status", [(0, 16, 16, 1), (4, 24, 16, 2), (4, 16, 24, 2), (4, 16, 2 ** 31, 1)])
+def test_qgemm_s32_shape_rules(lib, M, N, K, status):
+    assert lib.aria_qgemm_s32(M, N, K, OK_PTR, OK_PTR, OK_PTR, None) == status
+
+
+@pytest.mark.parametrize("M,K,status", [(0, 16, 1), (4, 0, 1), (4, 24, 2), (2 ** 31, 16, 1)])
+def test_act_quant_shape_rules(lib, M, K, status):
+    assert lib.aria_act_quant(OK_PTR, M, K, OK_PTR, OK_PTR, None) == status
+
+
+@pytest.mark.parametrize("fmt,group,N,K,status", [
+    (1, 0, 16, 24, 2),    # q8 pack: K % 16
+    (2, 32, 16, 48, 2),   # q4 pack: K % 32
+    (2, 64, 16, 64, 2),   # q4 pack: group 32 only
+    (1, 0, 0, 16, 1),     # N < 1
+])
+def test_qpack_shape_rules(lib, fmt, group, N, K, status):
+    assert lib.aria_qpack(fmt, group, OK_PTR, N, K, OK_PTR, OK_PTR, None) == status
