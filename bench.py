@@ -49,12 +49,19 @@ WORKLOAD = ("layer-sequence replay: 24 blocks x {qkv 1536->4608, out 1536->1536,
 # ----------------------------------------------------------------- helpers --
 
 def kernel_source_sha256():
+    """Hash of the CUDA sources' code: comments and whitespace are stripped,
+    so the traffic record stays valid across comment-only edits and goes
+    stale on any change to the code."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "int8_int4_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            t = fh.read()
+        t = re.sub(r"/\*.*?\*/", " ", t, flags=re.S)
+        t = re.sub(r"//[^\n]*", " ", t)
+        h.update(os.path.basename(f).encode() + b"\0" + " ".join(t.split()).encode() + b"\0")
     return h.hexdigest()
 
 

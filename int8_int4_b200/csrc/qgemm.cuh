@@ -10,23 +10,28 @@
 // without padding the token dimension to 128. Both operands are K-major in
 // the 128-byte swizzled shared-memory layout.
 //
-// Persistent, warp-specialised CTA (one per SM):
-//   warp 0       TMA producer of weight tiles (raw packed bytes for q8/q4, the
-//                int8 A operand itself for W8A8)
-//   warp 1       TMEM allocator (two accumulator buffers) and the single-thread
-//                tcgen05.mma issuer
-//   warp 2       TMA producer of activation tiles
+// Persistent, warp-specialised CTA (one per SM). The producer and MMA roles
+// run as converged warps: every lane waits on the barriers, one lane issues
+// (TMA by lane 0, tcgen05.mma / commit by elect.sync), which keeps the issue
+// loops on the uniform datapath.
+//   warp 0       TMA producer of weight tiles (raw packed bytes for q8/q4; for
+//                W8A8 the int8 weight and activation tiles of each stage). The
+//                first ring of weight tiles is loaded before the wait on the
+//                preceding kernel (programmatic dependent launch).
+//   warp 1       TMEM allocator (two accumulator buffers) and MMA issuer
+//   warp 2       q8/q4: TMA producer of activation tiles
 //   warps 4..7   epilogue: TMEM -> registers -> scale, bias, steer -> fp16 ->
 //                transposed through shared memory -> coalesced 16-byte stores;
 //                overlaps the next tile's mainloop through the second
 //                accumulator buffer (W8A8 uses warps 8..11 for it as well)
-//   warps 8..11  q8/q4 only: dequantise raw weights into fp16 A tiles (one
-//                weight row per thread; exact int8 -> fp16; fp16 code*scale for q4)
+//   warps 8..11  q8/q4: dequantise raw weights into fp16 A tiles (one weight
+//                row per thread; exact int8 -> fp16; fp16 code*scale for q4);
+//                they take part in the epilogue of the CTA's last tile
 // Rings of shared-memory stages with mbarriers connect the roles; every wait
 // is bounded. Split-K (few output tiles): a cluster of S CTAs shares one tile,
-// each taking a contiguous K range, and partial accumulators are summed
-// through distributed shared memory in fixed rank order (deterministic, no
-// global scratch).
+// each taking a contiguous K range; all warps then sum the partial
+// accumulators through distributed shared memory in fixed rank order
+// (deterministic, no global scratch).
 #pragma once
 
 #include <cuda_fp16.h>
