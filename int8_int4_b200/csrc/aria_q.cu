@@ -221,8 +221,9 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
 }
 
 // programmatic dependent launch: the kernel may start while the previous
-// kernel in the stream drains; it waits (griddepcontrol.wait) before touching
-// global memory
+// kernel in the stream drains; it waits (griddepcontrol.wait) before reading
+// anything that kernel may write (the GEMM's packed weights are the one
+// exception, see the stream-order note of aria_qgemm in the header)
 void set_pdl(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr) {
   attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
