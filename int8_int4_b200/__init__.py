@@ -95,6 +95,50 @@ def _group(fmt: str, group):
     return (32 if fmt == "q4" else 0) if group is None else int(group)
 
 
+def _expect(t, name: str, shape, dtype):
+    """Shape and dtype of an argument (checked before anything reaches the device:
+    the C ABI takes raw pointers and cannot see a too-small buffer)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def check_gemm_args(fmt: str, X, Wq, scales, sx=None, bias=None, steer_vec=None, out=None):
+    """The tensors of one GEMM call agree with each other and with the format
+    (include/aria_q.h): X [M,K] (fp16; int8 for W8A8), Wq [N,K] int8 (q8, W8A8)
+    or [N,K/2] uint8 (q4), scales fp32 [N] (q8, W8A8) or fp16 [N,K/32] (q4),
+    sx fp32 [M] (W8A8 only), bias fp16 [N], steer_vec fp32 [N], out fp16 [M,N].
+    Returns (M, N, K)."""
+    if fmt not in FORMATS:
+        raise ValueError(f"unknown format {fmt!r}")
+    if X.dim() != 2 or Wq.dim() != 2:
+        raise ValueError("X and Wq must be 2-D")
+    M, K = X.shape
+    N = Wq.shape[0]
+    _expect(X, "X", (M, K), torch.int8 if fmt == "w8a8" else torch.float16)
+    if fmt == "q4":
+        if K % 32:
+            raise ValueError("q4 needs K % 32 == 0")
+        _expect(Wq, "Wq", (N, K // 2), torch.uint8)
+        _expect(scales, "scales", (N, K // 32), torch.float16)
+    else:
+        _expect(Wq, "Wq", (N, K), torch.int8)
+        _expect(scales, "scales", (N,), torch.float32)
+    if fmt == "w8a8":
+        if sx is None:
+            raise ValueError("w8a8 needs sx")
+        _expect(sx, "sx", (M,), torch.float32)
+    elif sx is not None:
+        raise ValueError("sx is for w8a8 only")
+    _expect(bias, "bias", (N,), torch.float16)
+    _expect(steer_vec, "steer_vec", (N,), torch.float32)
+    _expect(out, "out", (M, N), torch.float16)
+    return M, N, K
+
+
 def qpack_size(fmt: str, N: int, K: int, group=None):
     wb, sb = ctypes.c_size_t(), ctypes.c_size_t()
     _check(load_library().aria_qpack_size(FORMATS[fmt], _group(fmt, group), N, K,
@@ -124,6 +168,8 @@ def act_quant(X: torch.Tensor, out=None, stream=None):
     Xq, sx = out if out is not None else (
         torch.empty(M, K, dtype=torch.int8, device=X.device),
         torch.empty(M, dtype=torch.float32, device=X.device))
+    _expect(Xq, "Xq", (M, K), torch.int8)
+    _expect(sx, "sx", (M,), torch.float32)
     _check(load_library().aria_act_quant(_dev(X, "X", torch.float16), M, K,
                                          _dev(Xq, "Xq", torch.int8), _dev(sx, "sx", torch.float32),
                                          _stream(stream)))
@@ -133,11 +179,8 @@ def act_quant(X: torch.Tensor, out=None, stream=None):
 def qgemm(fmt: str, X: torch.Tensor, Wq: torch.Tensor, scales: torch.Tensor, sx=None,
           bias=None, steer_vec=None, alpha: float = 0.0, group=None, out=None, stream=None):
     """Y [M,N] fp16 = X . dequant(W)^T + bias + alpha*v (see include/aria_q.h)."""
-    M, K = X.shape
-    N = Wq.shape[0]
+    M, N, K = check_gemm_args(fmt, X, Wq, scales, sx, bias, steer_vec, out)
     Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=X.device)
-    if tuple(Y.shape) != (M, N) or Y.dtype != torch.float16:
-        raise ValueError("out must be fp16 [M, N]")
     xdt = torch.int8 if fmt == "w8a8" else torch.float16
     _check(load_library().aria_qgemm(
         FORMATS[fmt], _group(fmt, group), M, N, K, _dev(X, "X", xdt),
@@ -151,7 +194,9 @@ def qgemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out=None, stream=None):
     """Raw int32 accumulators C [M,N] = Xq . Wq^T on the integer tensor cores."""
     M, K = Xq.shape
     N = Wq.shape[0]
+    _expect(Wq, "Wq", (N, K), torch.int8)
     C = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xq.device)
+    _expect(C, "out", (M, N), torch.int32)
     _check(load_library().aria_qgemm_s32(M, N, K, _dev(Xq, "Xq", torch.int8),
                                          _dev(Wq, "Wq", torch.int8), _dev(C, "out", torch.int32),
                                          _stream(stream)))

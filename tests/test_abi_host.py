@@ -131,3 +131,53 @@ def test_act_quant_shape_rules(lib, M, K, status):
 ])
 def test_qpack_shape_rules(lib, fmt, group, N, K, status):
     assert lib.aria_qpack(fmt, group, OK_PTR, N, K, OK_PTR, OK_PTR, None) == status
+
+
+def _args(fmt, M=8, N=32, K=256):
+    import torch
+    X = torch.zeros(M, K, dtype=torch.int8 if fmt == "w8a8" else torch.float16)
+    if fmt == "q4":
+        Wq, sc = torch.zeros(N, K // 2, dtype=torch.uint8), torch.zeros(N, K // 32, dtype=torch.float16)
+    else:
+        Wq, sc = torch.zeros(N, K, dtype=torch.int8), torch.zeros(N, dtype=torch.float32)
+    sx = torch.zeros(M, dtype=torch.float32) if fmt == "w8a8" else None
+    return dict(X=X, Wq=Wq, scales=sc, sx=sx, bias=torch.zeros(N, dtype=torch.float16),
+                steer_vec=torch.zeros(N, dtype=torch.float32), out=torch.zeros(M, N, dtype=torch.float16))
+
+
+@pytest.mark.parametrize("fmt", ["q8", "q4", "w8a8"])
+def test_binding_accepts_consistent_arguments(fmt):
+    assert aq.check_gemm_args(fmt, **_args(fmt)) == (8, 32, 256)
+    a = _args(fmt)
+    a.update(bias=None, steer_vec=None, out=None)
+    assert aq.check_gemm_args(fmt, **a) == (8, 32, 256)
+
+
+@pytest.mark.parametrize("fmt,field,bad", [
+    ("q8", "Wq", ("shape", (32, 128))),          # packed for another K: the kernel would read past it
+    ("q8", "scales", ("shape", (16,))),
+    ("q8", "X", ("dtype", "int8")),
+    ("q4", "Wq", ("shape", (32, 256))),          # a q8 pack passed as q4
+    ("q4", "scales", ("dtype", "float32")),
+    ("w8a8", "X", ("dtype", "float16")),          # not quantised
+    ("w8a8", "sx", ("shape", (4,))),
+    ("w8a8", "sx", ("none", None)),
+    ("q8", "sx", ("extra", None)),
+    ("q8", "bias", ("shape", (16,))),
+    ("q4", "steer_vec", ("dtype", "float16")),
+    ("w8a8", "out", ("shape", (8, 16))),
+])
+def test_binding_rejects_inconsistent_arguments(fmt, field, bad):
+    import torch
+    a = _args(fmt)
+    kind, val = bad
+    if kind == "shape":
+        a[field] = torch.zeros(val, dtype=a[field].dtype)
+    elif kind == "dtype":
+        a[field] = a[field].to(getattr(torch, val))
+    elif kind == "none":
+        a[field] = None
+    elif kind == "extra":
+        a[field] = torch.zeros(8, dtype=torch.float32)
+    with pytest.raises((ValueError, TypeError)):
+        aq.check_gemm_args(fmt, **a)
