@@ -361,3 +361,73 @@ def test_zero_inputs_give_bias():
     assert not Xq.any() and not sx.any()
     Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx, bias=b)
     assert torch.equal(Y.float(), b.float().expand(M, N))
+
+
+# --------------------------------------- the replay's launch configuration --
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_dependent_chain_in_replay_launch_configuration(graph):
+    """The replay's launch configuration -- back-to-back calls on one stream,
+    each kernel allowed to start before its predecessor has finished
+    (programmatic dependent launch), captured in one CUDA graph as bench.py
+    does -- with each call reading the previous call's output: q8
+    (1536 -> 6144), per-token activation quantisation of that output, W8A8
+    (6144 -> 1536, steered), q4 (1536 -> 4608), at M = 432. Each stage is
+    checked against the oracle on the input the GPU actually gave it, and the
+    chain runs three times with new activations, so a kernel that read its
+    input before its predecessor had written it would be computed from the
+    previous run's values."""
+    M, d, f = 432, 1536, 6144
+    key = "gpu/chain"
+    q1, s1 = aq.qpack("q8", synthetic.weight(f"{key}/up", f, d).cuda())
+    q2, s2 = aq.qpack("q8", synthetic.weight(f"{key}/down", d, f).cuda())
+    p3, t3 = aq.qpack("q4", synthetic.weight(f"{key}/qkv", 3 * d, d, outlier_frac=0.001).cuda())
+    v = synthetic.steer_vec(key, d)
+    vd = v.cuda()
+    X0 = torch.empty(M, d, dtype=torch.float16, device="cuda")
+    y1 = torch.empty(M, f, dtype=torch.float16, device="cuda")
+    xq = torch.empty(M, f, dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    y2 = torch.empty(M, d, dtype=torch.float16, device="cuda")
+    y3 = torch.empty(M, 3 * d, dtype=torch.float16, device="cuda")
+    st = torch.cuda.Stream()
+
+    def chain():
+        aq.qgemm("q8", X0, q1, s1, out=y1, stream=st)
+        aq.act_quant(y1, out=(xq, sx), stream=st)
+        aq.qgemm("w8a8", xq, q2, s2, sx=sx, steer_vec=vd, alpha=0.3, out=y2, stream=st)
+        aq.qgemm("q4", y2, p3, t3, out=y3, stream=st)
+
+    g = None
+    if graph:
+        X0.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(st):
+            chain()                      # eager once: first-call set-up outside capture
+            st.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                chain()
+        torch.cuda.synchronize()
+    w1, sw1 = q1.cpu().numpy(), s1.cpu().numpy()
+    w2, sw2 = q2.cpu().numpy(), s2.cpu().numpy()
+    w3, sw3 = p3.cpu().numpy(), t3.cpu().numpy().view(np.uint16)
+    rows = sample_rows(M, 12)
+    for r in range(3):
+        X0.copy_(synthetic.activation(f"{key}/x{r}", M, d).cuda())
+        torch.cuda.synchronize()
+        if g is not None:
+            g.replay()
+        else:
+            chain()
+        torch.cuda.synchronize()
+        x0, h1, h2, h3 = (f16np(t) for t in (X0, y1, y2, y3))
+        check_wo(h1[rows], oracle.wo_ref("q8", x0, w1, sw1, rows=rows))
+        rq, rs = oracle.act_quant(h1)
+        assert np.array_equal(xq.cpu().numpy(), rq), r
+        assert np.array_equal(sx.cpu().numpy().view(np.uint32), rs.view(np.uint32)), r
+        ref2 = oracle.w8a8(h1, w2, sw2, None, v.numpy(), 0.3, rows=rows)
+        assert np.array_equal(h2.view(np.uint16)[rows], ref2), r
+        check_wo(h3[rows], oracle.wo_ref("q4", h2, w3, sw3, rows=rows))
+    del g
+    aq.device_status()
