@@ -431,3 +431,53 @@ def test_dependent_chain_in_replay_launch_configuration(graph):
         check_wo(h3[rows], oracle.wo_ref("q4", h2, w3, sw3, rows=rows))
     del g
     aq.device_status()
+
+
+def test_bench_replay_outputs_match_oracle():
+    """bench.py's own workload and launches: bench.Replay's CUDA graphs (24
+    blocks x 4 linears x 8 steps per precision at M = 432, steering on block
+    12's out-projection), replayed precision by precision; then sampled
+    outputs of blocks 0, 12 and 23 against the oracle: q8 and q4 within the
+    weight-only tolerance, W8A8 bit-exact."""
+    import bench
+    rep = bench.Replay(torch.device("cuda", torch.cuda.current_device()))
+    rep.capture()
+    rows = sample_rows(bench.M, 4)
+    blocks = (0, synthetic.REPLAY_STEER_BLOCK, bench.BLOCKS - 1)
+    v = rep.steer.cpu().numpy()
+
+    def steer(b, name):
+        on = b == synthetic.REPLAY_STEER_BLOCK and name == "out"
+        return (v, synthetic.REPLAY_ALPHA) if on else (None, 0.0)
+
+    def replay(*kinds):
+        with torch.cuda.stream(rep.stream):
+            for kind in kinds:
+                rep.graphs[kind].replay()
+        torch.cuda.synchronize()
+
+    replay("q8")
+    for b in blocks:
+        for name, k, n in bench.LINEARS:
+            x = rep.x_host[b, name].numpy()
+            Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
+            vv, a = steer(b, name)
+            check_wo(f16np(rep.y[b, name])[rows], oracle.wo_ref("q8", x, Wq, sw, None, vv, a, rows=rows))
+    replay("act_quant", "w8a8_gemm")
+    for b in blocks:
+        for name, k, n in bench.LINEARS:
+            x = rep.x_host[b, name].numpy()
+            Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
+            vv, a = steer(b, name)
+            ref = oracle.w8a8(x, Wq, sw, None, vv, a, rows=rows)
+            assert np.array_equal(f16np(rep.y[b, name]).view(np.uint16)[rows], ref), (b, name)
+    replay("q4")
+    for b in blocks:
+        for name, k, n in bench.LINEARS:
+            x = rep.x_host[b, name].numpy()
+            P, S = rep.q4[b, name]
+            vv, a = steer(b, name)
+            ref = oracle.wo_ref("q4", x, P.cpu().numpy(), S.cpu().numpy().view(np.uint16), None, vv, a,
+                                rows=rows)
+            check_wo(f16np(rep.y[b, name])[rows], ref)
+    rep.aq.device_status(rep.stream)
