@@ -64,6 +64,8 @@ def sample_rows(M, k, seed=0):
 def test_pack_q8_bit_exact(N, K):
     W = synthetic.weight(f"gpu/pq8/{N}x{K}", N, K, outlier_frac=0.001)
     W[1] = 0                                   # an all-zero channel
+    t = 2.0 ** -24                             # a channel of fp16 subnormals
+    W[2] = torch.from_numpy(((np.arange(K) % 23) - 11) * t).to(torch.float16)
     Wq, s = aq.qpack("q8", W.cuda())
     rq, rs = oracle.pack_q8(W.numpy())
     assert np.array_equal(Wq.cpu().numpy(), rq)
@@ -74,6 +76,11 @@ def test_pack_q8_bit_exact(N, K):
 def test_pack_q4_bit_exact(N, K):
     W = synthetic.weight(f"gpu/pq4/{N}x{K}", N, K, outlier_frac=0.001)
     W[0, :32] = 0                              # an all-zero group
+    t = 2.0 ** -24                             # groups whose scale is an fp16 subnormal:
+    W[1, :32] = 0
+    W[1, 0], W[1, 3] = 10 * t, -2 * t          # s16 = 1 step, the code of 10 clamps to 7
+    W[1, 32:64] = 0
+    W[1, 37], W[1, 38] = 3 * t, -3 * t         # s16 rounds to 0: every code 0
     P, S = aq.qpack("q4", W.cuda())
     rp, rs = oracle.pack_q4(W.numpy())
     assert np.array_equal(P.cpu().numpy(), rp)

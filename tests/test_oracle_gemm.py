@@ -104,6 +104,19 @@ def test_w8a8_out_exact_rational(with_bias, with_steer):
             assert Y[m, n] == _half_rne_exact(t), (m, n)
 
 
+def test_w8a8_rows_subset_matches_full():
+    """Sampled rows (as the GPU tests use them) give the rows of the full
+    result: each output row takes the token scale of its own X row."""
+    M, N, K = 11, 48, 256
+    W = synthetic.weight("pin/w8a8rows/W", N, K).numpy()
+    X = synthetic.activation("pin/w8a8rows", M, K, outlier_channel_frac=0.01).numpy()
+    X[4] *= 8                                  # token scales that differ a lot
+    Wq, sw = oracle.pack_q8(W)
+    full = oracle.w8a8(X, Wq, sw)
+    rows = [9, 0, 4, 7]
+    assert np.array_equal(oracle.w8a8(X, Wq, sw, rows=rows), full[rows])
+
+
 def test_w8a8_close_to_unquantised_product():
     """|acc*sx*sw - x.w| <= sum_k (|x|*sw/2 + |w|*sx/2 + sx*sw/4) (plus fp32
     quotient slack): pins operand order, scale indexing and the int GEMM."""
