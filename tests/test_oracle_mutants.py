@@ -47,6 +47,8 @@ MUTANTS = [
     ("q4 reference code offset", "double w = (double)(nib - 8) * orc_half_to_double(S[n * G + k / 32]);",
      "double w = (double)(nib - 7) * orc_half_to_double(S[n * G + k / 32]);"),
     ("q4 clamp at 8", "if (r > 7.0f) r = 7.0f;", "if (r > 8.0f) r = 8.0f;"),
+    ("q4 clamp at -8", "if (r < -7.0f) r = -7.0f;", "if (r < -8.0f) r = -8.0f;"),
+    ("fp16 NaN encoded as infinity", "return (uint16_t)(sign | 0x7e00);", "return (uint16_t)(sign | 0x7c00);"),
     ("q4 zero scale not special", "if (sf != 0.0f) {", "if (sf != -1.0f) {"),
     ("W8A8 token scale of the output row", "double smx = (double)sx[pick(rows, i)];",
      "double smx = (double)sx[i];"),

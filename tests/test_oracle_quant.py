@@ -155,18 +155,18 @@ def test_q4_subnormal_scales():
     """Groups whose scale falls in the fp16 subnormal range, worked by hand
     (2^-24 is the smallest fp16 step):
     - absmax 10 * 2^-24: absmax / 7 = 1.43 steps rounds to s16 = 1 step, so
-      the quotient 10 is clamped to code 7 (nibble 15), not 8 or 10;
+      the quotients +-10 are clamped to codes +-7 (nibbles 15 and 1);
     - absmax 3 * 2^-24: absmax / 7 = 0.43 steps rounds to s16 = 0, and a zero
       scale gives code 0 (nibble 8) for every element, not +-7."""
     t = 2.0 ** -24
     W = np.zeros((2, 32), np.float64)
-    W[0, 0], W[0, 3] = 10 * t, -2 * t
+    W[0, 0], W[0, 3], W[0, 9] = 10 * t, -2 * t, -10 * t
     W[1, 5], W[1, 6] = 3 * t, -3 * t
     P, S = oracle.pack_q4(W.astype(np.float16))
     assert S[0, 0] == 0x0001 and S[1, 0] == 0x0000
     nib = np.stack([P & 0x0F, P >> 4], axis=-1).reshape(2, 32)
     expect0 = np.full(32, 8)
-    expect0[0], expect0[3] = 15, 8 - 2
+    expect0[0], expect0[3], expect0[9] = 15, 8 - 2, 1
     assert np.array_equal(nib[0], expect0)
     assert np.all(nib[1] == 8)
 
