@@ -78,7 +78,7 @@ def test_pack_q4_bit_exact(N, K):
     W[0, :32] = 0                              # an all-zero group
     t = 2.0 ** -24                             # groups whose scale is an fp16 subnormal:
     W[1, :32] = 0
-    W[1, 0], W[1, 3] = 10 * t, -2 * t          # s16 = 1 step, the code of 10 clamps to 7
+    W[1, 0], W[1, 3], W[1, 9] = 10 * t, -2 * t, -10 * t   # s16 = 1 step: +-10 clamp to +-7
     W[1, 32:64] = 0
     W[1, 37], W[1, 38] = 3 * t, -3 * t         # s16 rounds to 0: every code 0
     P, S = aq.qpack("q4", W.cuda())
