@@ -104,6 +104,20 @@ def test_w8a8_out_exact_rational(with_bias, with_steer):
             assert Y[m, n] == _half_rne_exact(t), (m, n)
 
 
+def test_w8a8_out_single_rounding_near_midpoints():
+    """Worked by hand at 2048..2052, where fp16 steps by 2: 2049 and 2051 are
+    exact midpoints (ties go to the even significand: 2048, 2052); 2049 plus
+    a bias of 2^-14 lies just above the midpoint and must round up to 2050.
+    Rounding through fp32 first would land on 2049.0 and then tie down to
+    2048, so this pins one rounding of the fp64 value."""
+    C = np.array([[2049, 2051, 2049]], np.int32)
+    sx = np.array([1.0], np.float32)
+    sw = np.array([1.0, 1.0, 1.0], np.float32)
+    b = np.array([0.0, 0.0, 2.0 ** -14], np.float16)
+    Y = oracle.w8a8_out(C, sx, sw, b)
+    assert list(Y[0]) == [0x6800, 0x6802, 0x6801]
+
+
 def test_w8a8_rows_subset_matches_full():
     """Sampled rows (as the GPU tests use them) give the rows of the full
     result: each output row takes the token scale of its own X row."""

@@ -48,6 +48,8 @@ MUTANTS = [
      "double w = (double)(nib - 7) * orc_half_to_double(S[n * G + k / 32]);"),
     ("q4 clamp at 8", "if (r > 7.0f) r = 7.0f;", "if (r > 8.0f) r = 8.0f;"),
     ("q4 clamp at -8", "if (r < -7.0f) r = -7.0f;", "if (r < -8.0f) r = -8.0f;"),
+    ("W8A8 output rounded through fp32", "Y[i * N + n] = orc_double_to_half(epi_terms(n, bias, v, alpha, y));",
+     "Y[i * N + n] = orc_double_to_half((double)(float)epi_terms(n, bias, v, alpha, y));"),
     ("fp16 NaN encoded as infinity", "return (uint16_t)(sign | 0x7e00);", "return (uint16_t)(sign | 0x7c00);"),
     ("q4 zero scale not special", "if (sf != 0.0f) {", "if (sf != -1.0f) {"),
     ("W8A8 token scale of the output row", "double smx = (double)sx[pick(rows, i)];",
