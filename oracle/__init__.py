@@ -11,7 +11,8 @@ Audio Generation" (aria project page): "What aria is" (weights packed from
 fp16 to 8 or 4 bits, the fp16 copy released), "Results" (the fp16 / q8 /
 W8A8 / q4 table; W8A8 is 8-bit arithmetic on integer tensor cores) and
 "Steering is real" (a direction added at one block, bit-identical at
-alpha = 0).
+alpha = 0). The unquantised fp16 rung of the "Results" table has a reference
+too (``f16_ref``).
 """
 from __future__ import annotations
 
@@ -62,6 +63,7 @@ def _load():
                 "orc_w8a8_out": ([P, P, P, I64, I64, P, I64, P, P, F32, P], None),
                 "orc_wo_q8_ref": ([P, P, P, I64, I64, I64, P, I64, P, P, F32, P], None),
                 "orc_wo_q4_ref": ([P, P, P, I64, I64, I64, P, I64, P, P, F32, P], None),
+                "orc_f16_ref": ([P, P, I64, I64, I64, P, I64, P, P, F32, P], None),
             }
             for name, (args, res) in sigs.items():
                 fn = getattr(lib, name)
@@ -256,4 +258,21 @@ def wo_ref(fmt, X, Wq, scales, bias=None, v=None, alpha=0.0, rows=None) -> np.nd
                           _ptr(b), _ptr(vv), float(alpha), _ptr(Y))
     else:
         raise ValueError(fmt)
+    return Y
+
+
+def f16_ref(X, W, bias=None, v=None, alpha=0.0, rows=None) -> np.ndarray:
+    """Unquantised fp16 reference ("Results": the fp16 column) in fp64, not
+    rounded: X @ W^T + bias + alpha*v with X [M,K] and W [N,K] fp16."""
+    X = _h(X)
+    W = _h(W)
+    M, K = X.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    r, R = _rows(rows, M)
+    Y = np.empty((R, N), np.float64)
+    _load().orc_f16_ref(_ptr(X), _ptr(W), M, N, K, _ptr(r), R,
+                        _ptr(_h(bias) if bias is not None else None), _ptr(_c(v, np.float32)),
+                        float(alpha), _ptr(Y))
     return Y

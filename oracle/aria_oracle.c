@@ -23,6 +23,9 @@
  *          y = fp16_rn(acc*s_x[m]*s_w[n] + bias[n] + alpha*v[n]) in fp64.
  *   weight-only (q8, q4): y_ref = sum_k X[m,k]*q[n,k]*s + bias[n] + alpha*v[n]
  *          in fp64, NOT rounded (the fp16 output is compared with tolerance).
+ *   fp16 : the unquantised rung of the "Results" precision table,
+ *          y_ref = sum_k X[m,k]*W[n,k] + bias[n] + alpha*v[n] in fp64, NOT
+ *          rounded (compared with the same tolerance as weight-only).
  * Every division is the IEEE fp32 quotient, rounded once; every rounding to
  * an integer is round-half-even (nearbyint under the default rounding mode).
  * An all-zero row / group / token gets scale 0 and codes 0.
@@ -294,6 +297,26 @@ void orc_wo_q4_ref(const uint16_t *X, const uint8_t *P, const uint16_t *S, int64
                 double w = (double)(nib - 8) * orc_half_to_double(S[n * G + k / 32]);
                 y += orc_half_to_double(x[k]) * w;
             }
+            Yref[i * N + n] = epi_terms(n, bias, v, alpha, y);
+        }
+    }
+}
+
+/* fp16 (unquantised) reference, fp64 and unrounded (the fp16 column of the
+ * "Results" precision table):
+ * Yref[i,n] = sum_k X[rows[i],k] * W[n,k] + bias[n] + alpha*v[n]. */
+void orc_f16_ref(const uint16_t *X, const uint16_t *W, int64_t M, int64_t N, int64_t K,
+                 const int64_t *rows, int64_t n_rows, const uint16_t *bias, const float *v,
+                 float alpha, double *Yref)
+{
+    int64_t R = rows ? n_rows : M;
+    for (int64_t i = 0; i < R; ++i) {
+        const uint16_t *x = X + pick(rows, i) * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint16_t *w = W + n * K;
+            double y = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                y += orc_half_to_double(x[k]) * orc_half_to_double(w[k]);
             Yref[i * N + n] = epi_terms(n, bias, v, alpha, y);
         }
     }

@@ -204,3 +204,60 @@ def test_epilogue_special_cases():
     y0 = oracle.wo_ref("q8", X, Wq, sw, b)
     y1 = oracle.wo_ref("q8", X, Wq, sw, b, v, 0.3)
     assert np.allclose(y1 - y0, np.float64(np.float32(0.3)) * v.astype(np.float64), rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------- the unquantised rung ---
+# "Results" (aria project page): the fp16 column of the precision table is
+# the transformer with its weights left in fp16. Its reference is the plain
+# product in fp64, unrounded.
+
+def test_f16_ref_matches_numpy_matmul():
+    M, N, K = 7, 40, 384
+    W = synthetic.weight("pin/f16/W", N, K, outlier_frac=0.001).numpy()
+    X = synthetic.activation("pin/f16", M, K).numpy()
+    b = synthetic.bias("pin/f16", N).numpy()
+    v = synthetic.steer_vec("pin/f16", N).numpy()
+    Y = oracle.f16_ref(X, W, b, v, 0.3)
+    a32 = np.float64(np.float32(0.3))
+    ref = X.astype(np.float64) @ W.astype(np.float64).T + b.astype(np.float64) + a32 * v.astype(np.float64)
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+    rows = [6, 0, 2]
+    assert np.array_equal(oracle.f16_ref(X, W, b, v, 0.3, rows=rows), Y[rows])
+
+
+def test_f16_ref_exact_on_small_integers():
+    """Integer-valued operands (|x|, |w| <= 8): every product and partial sum
+    is an integer far below 2^53, so the fp64 result equals numpy's int64
+    matmul exactly, independent of summation order."""
+    rng = np.random.default_rng(3)
+    M, N, K = 5, 24, 300
+    xi = rng.integers(-8, 9, (M, K))
+    wi = rng.integers(-8, 9, (N, K))
+    Y = oracle.f16_ref(xi.astype(np.float16), wi.astype(np.float16))
+    assert np.array_equal(Y, (xi @ wi.T).astype(np.float64))
+
+
+def test_f16_ref_one_hot_reads_the_layout_back():
+    """X = e_k reads column k of W [N,K] (out x in), exactly: a transposed or
+    shifted index gives other values."""
+    N, K = 24, 40                              # N != K: a transposed read differs
+    W = synthetic.weight("pin/f16onehot/W", N, K).numpy()
+    X = np.zeros((K, K), np.float16)
+    X[np.arange(K), np.arange(K)] = 1
+    Y = oracle.f16_ref(X, W)
+    assert np.array_equal(Y, W.astype(np.float64).T)
+
+
+def test_f16_ref_epilogue_special_cases():
+    N, K = 32, 128
+    W = synthetic.weight("pin/f16epi/W", N, K).numpy()
+    b = synthetic.bias("pin/f16epi", N).numpy()
+    v = synthetic.steer_vec("pin/f16epi", N).numpy()
+    Z = np.zeros((3, K), np.float16)
+    assert np.array_equal(oracle.f16_ref(Z, W, b), np.tile(b.astype(np.float64), (3, 1)))
+    X = synthetic.activation("pin/f16epi", 4, K).numpy()
+    base = oracle.f16_ref(X, W, b)
+    assert np.array_equal(oracle.f16_ref(X, W, b, v, 0.0), base)
+    assert np.array_equal(oracle.f16_ref(X, W, b, None, 0.7), base)
+    y1 = oracle.f16_ref(X, W, b, v, 0.3)
+    assert np.allclose(y1 - base, np.float64(np.float32(0.3)) * v.astype(np.float64), rtol=0, atol=1e-12)

@@ -54,6 +54,12 @@ MUTANTS = [
     ("q4 zero scale not special", "if (sf != 0.0f) {", "if (sf != -1.0f) {"),
     ("W8A8 token scale of the output row", "double smx = (double)sx[pick(rows, i)];",
      "double smx = (double)sx[i];"),
+    ("fp16 reference reads W transposed", "y += orc_half_to_double(x[k]) * orc_half_to_double(w[k]);",
+     "y += orc_half_to_double(x[k]) * orc_half_to_double(W[k * N + n]);"),
+    ("fp16 reference drops the last k", "y += orc_half_to_double(x[k]) * orc_half_to_double(w[k]);",
+     "y += orc_half_to_double(x[k]) * orc_half_to_double(w[k]) * (double)(k + 1 < K);"),
+    ("fp16 reference weight row of the token", "const uint16_t *w = W + n * K;",
+     "const uint16_t *w = W + (n % 8) * K;"),
 ]
 
 
