@@ -8,12 +8,23 @@ down 6144->1536} at M = 432 tokens (2 CFG halves x 216 latent frames), 8
 denoising steps, at each of the three precisions, with the steering add
 (alpha = 0.3, unit-norm v) on block 12's out-projection. This is the shape of
 the pages' generation loop ("Results": 8 steps; "What aria is": the
-denoising loop replayed as one CUDA graph); weights are packed once at load,
-as on the pages, and the pack kernels are timed separately. Per precision
-one CUDA graph holds the 8-step loop (768 GEMM launches; W8A8 adds 768
-per-token activation quantisations in a graph of their own).
+denoising loop replayed as one CUDA graph; "Live steering while streaming":
+the steering strength lives inside the captured graph, here a device-side
+schedule read by the steered launch of each step). Weights are packed once
+at load, as on the pages. Per precision one CUDA graph holds the 8-step loop
+(768 GEMM launches; W8A8 adds 768 per-token activation quantisations).
+
+Beside the step, outside `value`: the unquantised fp16 rung of the
+precision ladder on the same replay, the steering on/off delta (the same
+graphs with the schedule set to 0), every per-shape case of the benchmark
+configurations (`per_config`: q8 d=1024 at M in {1,16,432}, W8A8 d=1536 at
+M in {432,4096} with its activation quantisation, q4 d=1536 at M in
+{1,8,432}, the fp16 rung, the packs), the end-to-end loop through host
+memory, and the CPU oracle.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep            # the per-shape cases only, one JSON line each
+    python bench.py --case q4 --shape 6144x1536 --m 432   # one case (ncu captures)
 
 N > 1 runs N independent replicas (one process per GPU, launched by torchrun),
 no collective on the data path; the timed region is bracketed by barriers
@@ -22,6 +33,7 @@ and the slowest rank's device time is reported. Rank 0 prints ONE JSON line.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import json
 import os
 import statistics
@@ -211,13 +223,22 @@ def bytes_w8a8(m, n, k, steer):
     return m * k + 4 * m + n * k + 4 * n + 2 * m * n + (4 * n if steer else 0)
 
 
+def bytes_f16(m, n, k, steer):
+    return 2 * n * k + 2 * m * k + 2 * m * n + (4 * n if steer else 0)
+
+
 def bytes_act_quant(m, k):
     return 3 * m * k + 4 * m
 
 
+def bytes_pack(fmt, n, k):
+    return 2 * n * k + (n * k + 4 * n if fmt == "q8" else n * k // 2 + 2 * n * (k // 32))
+
+
 def step_account():
     """ops and algorithmic bytes of one 8-step replay, per precision / kernel"""
-    acc = {"q8": [0.0, 0.0], "w8a8_gemm": [0.0, 0.0], "act_quant": [0.0, 0.0], "q4": [0.0, 0.0]}
+    acc = {"q8": [0.0, 0.0], "w8a8_gemm": [0.0, 0.0], "act_quant": [0.0, 0.0], "q4": [0.0, 0.0],
+           "f16": [0.0, 0.0]}
     for b in range(BLOCKS):
         for name, k, n in LINEARS:
             st = (b == synthetic.REPLAY_STEER_BLOCK and name == "out")
@@ -229,195 +250,263 @@ def step_account():
             acc["w8a8_gemm"][0] += o
             acc["w8a8_gemm"][1] += bytes_w8a8(M, n, k, st)
             acc["act_quant"][1] += bytes_act_quant(M, k)
+            acc["f16"][0] += o
+            acc["f16"][1] += bytes_f16(M, n, k, st)
     return {k: (v[0] * STEPS, v[1] * STEPS) for k, v in acc.items()}
+
+
+def roofs(peaks):
+    """Roofline denominators. A kernel timed inside the replay (a ~30 ms step
+    at full clocks, no power-cap throttling in the clock record) or alone in
+    a per-shape graph takes the burst GEMM figure; int8 is the fp16/bf16
+    figure times the nominal dense int8 : fp16 ratio (2)."""
+    f16 = peaks["bf16_tflops"]
+    return {"f16": f16, "i8": f16 * INT8_OVER_F16, "hbm": peaks["hbm_gbs"]}
+
+
+def roof_entry(ops, byts, seconds, tensor_peak, hbm):
+    """TOPS, GB/s, the binding roof (the larger ideal time) and the fraction
+    of it that this time reaches."""
+    d = {"us": seconds * 1e6, "gbs": byts / seconds / 1e9, "hbm_frac": byts / seconds / 1e9 / hbm}
+    if ops:
+        d["tops"] = ops / seconds / 1e12
+        d["tensor_frac"] = d["tops"] / tensor_peak
+        d["bound"] = "tensor" if ops / (tensor_peak * 1e12) >= byts / (hbm * 1e9) else "hbm"
+    else:
+        d["bound"] = "hbm"
+    d["frac"] = d["tensor_frac"] if d["bound"] == "tensor" else d["hbm_frac"]
+    return d
 
 
 # ------------------------------------------------------------- our arm ------
 
 class Replay:
-    """Device-resident workload and its CUDA graphs."""
+    """Device-resident workload and its CUDA graphs.
 
-    def __init__(self, dev):
+    Each precision has its own output buffers (the step's results stay
+    distinct), the fp16 rung keeps the unquantised weights, and the inputs
+    exist in `buffers` device copies so the end-to-end loop can copy the next
+    step's inputs while the current step computes. The steered launch of
+    step s reads its strength from `alpha[s]` (device memory)."""
+
+    ORDER = ("q8", "act_quant", "w8a8_gemm", "q4")       # the timed step
+    LAUNCHES_PER_STEP = len(ORDER) * STEPS * BLOCKS * len(LINEARS)
+
+    def __init__(self, dev, buffers=1, fp16=True):
         import int8_int4_b200 as aq
         self.aq = aq
         self.dev = dev
+        self.buffers = buffers
+        self.fp16 = fp16
         self.steer = synthetic.replay_steer().to(dev)
-        self.q8, self.q4, self.x, self.xq, self.y = {}, {}, {}, {}, {}
-        self.x_host = {}
+        self.alpha = torch.full((STEPS,), synthetic.REPLAY_ALPHA, dtype=torch.float32, device=dev)
+        self.q8, self.q4, self.w16, self.xq, self.x_host = {}, {}, {}, {}, {}
+        self.x = [dict() for _ in range(buffers)]
+        self.y = {k: {} for k in ("q8", "w8a8", "q4", "f16")}
         for b in range(BLOCKS):
             for name, k, n in LINEARS:
                 W = synthetic.replay_weight(b, name).to(dev)
                 self.q8[b, name] = aq.qpack("q8", W)
                 self.q4[b, name] = aq.qpack("q4", W)
-                del W                                   # the fp16 copy is released once packed
+                if fp16:
+                    self.w16[b, name] = W                 # the fp16 rung keeps its weights
+                del W                                     # the quantised rungs release theirs
                 xh = synthetic.replay_activation(b, name).pin_memory()
                 self.x_host[b, name] = xh
-                self.x[b, name] = xh.to(dev)
+                for i in range(buffers):
+                    self.x[i][b, name] = xh.to(dev)
                 self.xq[b, name] = (torch.empty(M, k, dtype=torch.int8, device=dev),
                                     torch.empty(M, dtype=torch.float32, device=dev))
-                self.y[b, name] = torch.empty(M, n, dtype=torch.float16, device=dev)
+                for prec in self.y:
+                    if prec != "f16" or fp16:
+                        self.y[prec][b, name] = torch.empty(M, n, dtype=torch.float16, device=dev)
         torch.cuda.synchronize()
 
-    def _steer(self, b, name):
+    def _steer(self, s, b, name):
         if b == synthetic.REPLAY_STEER_BLOCK and name == "out":
-            return dict(steer_vec=self.steer, alpha=synthetic.REPLAY_ALPHA)
+            return dict(steer_vec=self.steer, alpha_dev=self.alpha[s:s + 1])
         return {}
 
-    def launch(self, kind, stream):
+    def final_outputs(self, kinds=("q8", "w8a8", "q4")):
+        """The step's results: the last linear's output of each precision."""
+        return [self.y[k][BLOCKS - 1, LINEARS[-1][0]] for k in kinds]
+
+    def launch(self, kind, stream, buf=0):
         aq = self.aq
-        for _ in range(STEPS):
+        x = self.x[buf]
+        for s in range(STEPS):
             for b in range(BLOCKS):
                 for name, k, n in LINEARS:
                     key = (b, name)
                     if kind == "q8":
-                        aq.qgemm("q8", self.x[key], *self.q8[key], out=self.y[key], stream=stream,
-                                 **self._steer(b, name))
+                        aq.qgemm("q8", x[key], *self.q8[key], out=self.y["q8"][key], stream=stream,
+                                 **self._steer(s, b, name))
                     elif kind == "q4":
-                        aq.qgemm("q4", self.x[key], *self.q4[key], out=self.y[key], stream=stream,
-                                 **self._steer(b, name))
+                        aq.qgemm("q4", x[key], *self.q4[key], out=self.y["q4"][key], stream=stream,
+                                 **self._steer(s, b, name))
+                    elif kind == "f16":
+                        aq.qgemm("f16", x[key], self.w16[key], None, out=self.y["f16"][key],
+                                 stream=stream, **self._steer(s, b, name))
                     elif kind == "act_quant":
-                        aq.act_quant(self.x[key], out=self.xq[key], stream=stream)
+                        aq.act_quant(x[key], out=self.xq[key], stream=stream)
                     else:
                         xq, sx = self.xq[key]
-                        aq.qgemm("w8a8", xq, *self.q8[key], sx=sx, out=self.y[key], stream=stream,
-                                 **self._steer(b, name))
+                        aq.qgemm("w8a8", xq, *self.q8[key], sx=sx, out=self.y["w8a8"][key],
+                                 stream=stream, **self._steer(s, b, name))
+
+    def kinds(self):
+        return self.ORDER + (("f16",) if self.fp16 else ())
 
     def capture(self):
         self.stream = torch.cuda.Stream(self.dev)
+        self.copy_stream = torch.cuda.Stream(self.dev)
         self.graphs = {}
         with torch.cuda.stream(self.stream):
-            for kind in ("q8", "act_quant", "w8a8_gemm", "q4"):
+            for kind in self.kinds():
                 self.launch(kind, self.stream)   # eager once: first-call set-up outside capture
             self.stream.synchronize()
-            for kind in ("q8", "act_quant", "w8a8_gemm", "q4"):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=self.stream):
-                    self.launch(kind, self.stream)
-                self.graphs[kind] = g
+            for kind in self.kinds():
+                for buf in range(self.buffers if kind != "w8a8_gemm" else 1):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=self.stream):
+                        self.launch(kind, self.stream, buf)
+                    self.graphs[kind, buf] = g
         torch.cuda.synchronize()
         self.aq.device_status(self.stream)
 
-    ORDER = ("q8", "act_quant", "w8a8_gemm", "q4")
-    LAUNCHES_PER_STEP = 4 * STEPS * BLOCKS * len(LINEARS)
-
-    def run_step(self, events=None):
+    def run_step(self, events=None, buf=0, kinds=None):
         s = self.stream
+        kinds = self.ORDER if kinds is None else kinds
         with torch.cuda.stream(s):
-            for i, kind in enumerate(self.ORDER):
+            for i, kind in enumerate(kinds):
                 if events is not None:
                     events[i].record(s)
-                self.graphs[kind].replay()
+                self.graphs[kind, buf if kind != "w8a8_gemm" else 0].replay()
             if events is not None:
                 events[-1].record(s)
 
 
-def time_pack(dev, reps=3):
-    """pack kernels on block 0's four d=1536 weights, each timed alone after an
-    L2 flush; returns algorithmic GB/s per format"""
-    import int8_int4_b200 as aq
-    Ws = [synthetic.replay_weight(0, name).to(dev) for name, _, _ in LINEARS]
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    res = {}
-    for fmt in ("q8", "q4"):
-        tot_t, tot_b = 0.0, 0.0
-        for r in range(reps + 1):
-            for W in Ws:
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                aq.qpack(fmt, W)
-                e1.record()
-                e1.synchronize()
-                if r:                                  # first round is a warm-up
-                    n, k = W.shape
-                    tot_t += e0.elapsed_time(e1) * 1e-3
-                    tot_b += 2 * n * k + (n * k + 4 * n if fmt == "q8" else n * k // 2 + 2 * n * (k // 32))
-        res[fmt] = {"gbs": tot_b / tot_t / 1e9, "launches": 4 * reps}
-    del Ws, flush
-    return res
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_steps(rep, steps, ws, kinds=None):
+    """Device time of `steps` replays of `kinds`, bracketed by a barrier and a
+    synchronize on both sides; returns (total ms, per-kind ms lists)."""
+    kinds = Replay.ORDER if kinds is None else kinds
+    ev = [[_ev() for _ in range(len(kinds) + 1)] for _ in range(steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0, t1 = _ev(), _ev()
+    t0.record(rep.stream)
+    for s in range(steps):
+        rep.run_step(ev[s], kinds=kinds)
+    t1.record(rep.stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    seg = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) for i in range(len(kinds))]
+    return t0.elapsed_time(t1), seg
+
+
+def e2e_loop(rep, steps, out_host):
+    """End to end through host memory: every step copies all of its inputs
+    from pinned host memory (on a copy stream, into the input buffer the
+    previous step is not using) and reads its results back. Returns ms."""
+    cs, xs = rep.stream, rep.copy_stream
+    nb = rep.buffers
+    copied = [_ev() for _ in range(nb)]
+    done = [_ev() for _ in range(nb)]
+    start, end = _ev(), _ev()
+    start.record(xs)
+    for i in range(steps):
+        b = i % nb
+        with torch.cuda.stream(xs):
+            if i >= nb:
+                xs.wait_event(done[b])               # step i - nb has finished reading buffer b
+            for key, xh in rep.x_host.items():
+                rep.x[b][key].copy_(xh, non_blocking=True)
+            copied[b].record(xs)
+        cs.wait_event(copied[b])
+        rep.run_step(buf=b)
+        with torch.cuda.stream(cs):
+            for o, h in zip(rep.final_outputs(), out_host):
+                h.copy_(o, non_blocking=True)
+            done[b].record(cs)
+    end.record(cs)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def _gpu_bus_id(dev):
+    try:
+        return torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        try:
+            p = torch.cuda.get_device_properties(dev)
+            return f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        except Exception:
+            return None
 
 
 def run_ours(args, ws, rank):
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     dev = torch.device("cuda", torch.cuda.current_device())
     peaks, peak_src = load_peaks()
+    R = roofs(peaks)
     acct = step_account()
 
-    rep = Replay(dev)
+    rep = Replay(dev, buffers=2, fp16=not args.no_fp16)
     rep.capture()
     for _ in range(args.warmup):
         rep.run_step()
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    bus = None
-    try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
-    except Exception:
-        try:
-            p = torch.cuda.get_device_properties(dev)
-            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
-        except Exception:
-            bus = None
+    bus = _gpu_bus_id(dev)
     with ClockSampler(bus if isinstance(bus, str) else None) as clk:
-        barrier(ws)
-        torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(rep.stream)
-        for s in range(args.steps):
-            rep.run_step(ev[s])
-        t1.record(rep.stream)
-        torch.cuda.synchronize()
-        barrier(ws)
+        total_ms, seg_ms = time_steps(rep, args.steps, ws)
     clocks = clk.summary()
-    total_ms = t0.elapsed_time(t1)
-    seg_ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) for i in range(4)]
     rep.aq.device_status(rep.stream)
 
-    # ---- end to end: pinned host inputs -> device, the same graphs, result -> host
-    e2e_in = sum(t.numel() * t.element_size() for t in rep.x_host.values())
-    outs = [rep.y[BLOCKS - 1, "down"]]
-    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    e2e_out = sum(o.numel() * o.element_size() for o in outs)
-    for _ in range(max(1, args.warmup // 2)):
-        _e2e_step(rep, out_host)
-    torch.cuda.synchronize()
-    barrier(ws)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(rep.stream)
-    for _ in range(args.steps):
-        _e2e_step(rep, out_host)
-    a1.record(rep.stream)
-    torch.cuda.synchronize()
-    barrier(ws)
-    e2e_ms = a0.elapsed_time(a1)
+    # the steering on/off delta: the same graphs, the device schedule set to 0
+    rep.alpha.zero_()
+    off_ms, _ = time_steps(rep, args.steps, ws)
+    rep.alpha.fill_(synthetic.REPLAY_ALPHA)
+    # the fp16 rung of the precision ladder, same replay (outside `value`)
+    f16_ms = None
+    if rep.fp16:
+        for _ in range(max(1, args.warmup // 2)):
+            rep.run_step(kinds=("f16",))
+        f16_ms, _ = time_steps(rep, args.steps, ws, kinds=("f16",))
+    rep.aq.device_status(rep.stream)
 
-    total_ms, e2e_ms, *seg_ms = max_over_ranks([total_ms, e2e_ms, *seg_ms], ws)
-    pack = time_pack(dev) if rank == 0 else None
+    # ---- end to end: pinned host inputs -> device, the same graphs, results -> host
+    e2e_in = sum(t.numel() * t.element_size() for t in rep.x_host.values())
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in rep.final_outputs()]
+    e2e_out = sum(o.numel() * o.element_size() for o in out_host)
+    e2e_loop(rep, max(2, args.warmup), out_host)
+    barrier(ws)
+    e2e_ms = e2e_loop(rep, args.steps, out_host)
+    barrier(ws)
+    rep.aq.device_status(rep.stream)
+
+    vals = max_over_ranks([total_ms, e2e_ms, off_ms, f16_ms or 0.0, *seg_ms], ws)
+    total_ms, e2e_ms, off_ms, f16_ms_max, *seg_ms = vals
+    if f16_ms is not None:
+        f16_ms = f16_ms_max
 
     ops_step = acct["q8"][0] + acct["q4"][0] + acct["w8a8_gemm"][0]
     ms_per_step = total_ms / args.steps
     value = ops_step * ws / (ms_per_step * 1e-3) / 1e12
-    f16_peak = peaks["bf16_tflops_sustained"]
-    i8_peak = f16_peak * INT8_OVER_F16
-    hbm = peaks["hbm_gbs"]
-    kinds = {"q8": (0, f16_peak), "act_quant": (1, None), "w8a8_gemm": (2, i8_peak), "q4": (3, f16_peak)}
-    per = {}
+    hbm = R["hbm"]
+    kinds = {"q8": (0, R["f16"]), "act_quant": (1, None), "w8a8_gemm": (2, R["i8"]), "q4": (3, R["f16"])}
     launches = STEPS * BLOCKS * len(LINEARS)
+    per = {}
     for kind, (i, peak) in kinds.items():
         t = seg_ms[i] / args.steps * 1e-3
         ops, byts = acct[kind]
-        d = {"ms_per_step": seg_ms[i] / args.steps, "launches_per_step": launches,
-             "avg_launch_us": t / launches * 1e6, "hbm_gbs": byts / t / 1e9,
-             "hbm_frac": byts / t / 1e9 / hbm}
-        if ops:
-            d["tops"] = ops / t / 1e12
-            d["tensor_frac"] = d["tops"] / peak
-            # which roof binds at this shape: ideal time against each peak
-            d["bound"] = "tensor" if ops / (peak * 1e12) >= byts / (hbm * 1e9) else "hbm"
-        else:
-            d["bound"] = "hbm"
+        d = roof_entry(ops, byts, t, peak or 1.0, hbm)
+        d.update(ms_per_step=seg_ms[i] / args.steps, launches_per_step=launches,
+                 avg_launch_us=t / launches * 1e6)
         per[kind] = d
     per_precision = {
         "q8": per["q8"], "q4": per["q4"],
@@ -425,6 +514,13 @@ def run_ours(args, ws, rank):
                  "tops": acct["w8a8_gemm"][0] / ((seg_ms[1] + seg_ms[2]) / args.steps * 1e-3) / 1e12,
                  "gemm": per["w8a8_gemm"], "act_quant": per["act_quant"]},
     }
+    if f16_ms is not None:
+        t = f16_ms / args.steps * 1e-3
+        d = roof_entry(acct["f16"][0], acct["f16"][1], t, R["f16"], hbm)
+        d.update(ms_per_step=f16_ms / args.steps, launches_per_step=launches,
+                 avg_launch_us=t / launches * 1e6,
+                 note="the unquantised fp16 rung (\"Results\" table), timed after the step, not in value")
+        per_precision["f16"] = d
     dom = max(kinds, key=lambda k: seg_ms[kinds[k][0]])
     dd = per[dom]
     ops_l = acct[dom][0] / launches            # algorithmic work per launch (mean of 4 shapes)
@@ -440,8 +536,12 @@ def run_ours(args, ws, rank):
                       "act_quant": "row_quant_i8_kernel"}[dom]
     roof["traffic"], roof["traffic_source"] = measured_traffic(roof["kernel"], acct[dom][1] / launches)
     roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json "
-                           + ("bf16_tflops_sustained" if roof["bound"] == "tensor" else "hbm_gbs")
+                           + ("bf16_tflops (burst: the kernel runs inside a ~30 ms step at full clocks)"
+                              if roof["bound"] == "tensor" else "hbm_gbs")
                            + (" x 2 (nominal int8:fp16)" if dom == "w8a8_gemm" else ""))
+    if roof["bound"] == "tensor":
+        roof["frac_of_sustained"] = roof["achieved"] / (
+            peaks["bf16_tflops_sustained"] * (INT8_OVER_F16 if dom == "w8a8_gemm" else 1.0))
     roof["per_launch"] = {"ops": ops_l, "bytes": byt_l, "avg_us": t_l * 1e6}
 
     line = {
@@ -449,182 +549,248 @@ def run_ours(args, ws, rank):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16+i8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens": M, "blocks": BLOCKS, "denoise_steps": STEPS,
-                   "graphs": "one CUDA graph per precision holding the 8-step loop",
+                   "graphs": "one CUDA graph per precision holding the 8-step loop; the steered "
+                             "launch of step s reads alpha from a device schedule",
                    "l2": "inputs larger than L2: 680 MB q8 / 382 MB q4 weights and 221 MB of "
                          "activations cycle through each step",
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "per_precision": per_precision,
-        "pack_gbs": pack,
+        "steer_delta": {"steered_ms_per_step": ms_per_step, "unsteered_ms_per_step": off_ms / args.steps,
+                        "delta_ms_per_step": ms_per_step - off_ms / args.steps,
+                        "note": "the same captured graphs; the device alpha schedule set to 0 "
+                                "(the add is skipped) vs 0.3 on block 12's out-projection"},
         "roofline": roof,
         "gpu_launches": Replay.LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
         "e2e": {"value": ops_step * ws / (e2e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
                 "h2d_bytes_per_step": e2e_in, "d2h_bytes_per_step": e2e_out,
-                "ms_per_step": e2e_ms / args.steps},
+                "ms_per_step": e2e_ms / args.steps,
+                "note": "every step copies all 96 input activations from pinned host memory "
+                        "(double-buffered: the next step's copy overlaps this step's compute) and "
+                        "reads back each precision's final output; the other outputs are "
+                        "intermediates that a transformer consumes on the device"},
     }
+    if rank == 0 and not args.no_per_config:
+        line["per_config"] = run_cases(CONFIG_CASES, args.reps, R)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(rows=args.cpu_rows)
     return line
 
 
-def _e2e_step(rep, out_host):
-    s = rep.stream
-    with torch.cuda.stream(s):
-        for key, xh in rep.x_host.items():
-            rep.x[key].copy_(xh, non_blocking=True)
-    rep.run_step()
-    with torch.cuda.stream(s):
-        for o, h in zip([rep.y[BLOCKS - 1, "down"]], out_host):
-            h.copy_(o, non_blocking=True)
-
-
 # ------------------------------------------------------------- oracle arm --
 
-def cpu_sample(rows_per_gemm=8, linears=LINEARS, block=0, fmts=("q8", "w8a8", "q4")):
-    """One bounded sample of the workload through the oracle: for each
-    precision and each linear of one block, the whole pipeline (pack, act
-    quant where used, GEMM, epilogue) on `rows_per_gemm` token rows.
-    Returns (gemm ops counted like the GPU arm, seconds)."""
+def _cpu_pipeline(name, k, n, fmt, rows, block):
+    """One linear at one precision through the oracle: pack, act quant where
+    used, GEMM and epilogue on `rows` token rows. Returns (ops, seconds)."""
     import oracle
-    ops, t = 0.0, 0.0
-    rows = np.arange(rows_per_gemm)
-    for name, k, n in linears:
-        W = synthetic.replay_weight(block, name).numpy()
-        X = synthetic.replay_activation(block, name).numpy()
-        st = name == "out" and block == synthetic.REPLAY_STEER_BLOCK
-        v = synthetic.replay_steer().numpy() if st else None
-        a = synthetic.REPLAY_ALPHA if st else 0.0
-        for fmt in fmts:
-            t0 = time.perf_counter()
-            if fmt == "q4":
-                P, S = oracle.pack_q4(W)
-                oracle.wo_ref("q4", X[rows], P, S, None, v, a)
-            else:
-                Wq, sw = oracle.pack_q8(W)
-                if fmt == "q8":
-                    oracle.wo_ref("q8", X[rows], Wq, sw, None, v, a)
-                else:
-                    oracle.w8a8(X[rows], Wq, sw, None, v, a)
-            t += time.perf_counter() - t0
-            ops += gemm_ops(rows_per_gemm, n, k)
-    return ops, t
+    W = synthetic.replay_weight(block, name).numpy()
+    X = synthetic.replay_activation(block, name).numpy()
+    st = name == "out" and block == synthetic.REPLAY_STEER_BLOCK
+    v = synthetic.replay_steer().numpy() if st else None
+    a = synthetic.REPLAY_ALPHA if st else 0.0
+    r = np.arange(rows)
+    t0 = time.perf_counter()
+    if fmt == "q4":
+        P, S = oracle.pack_q4(W)
+        oracle.wo_ref("q4", X[r], P, S, None, v, a)
+    else:
+        Wq, sw = oracle.pack_q8(W)
+        if fmt == "q8":
+            oracle.wo_ref("q8", X[r], Wq, sw, None, v, a)
+        else:
+            oracle.w8a8(X[r], Wq, sw, None, v, a)
+    return gemm_ops(rows, n, k), time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except Exception:
+        return max(1, os.cpu_count() or 1)
+
+
+def cpu_sample(rows_per_gemm=8, linears=LINEARS, block=0, fmts=("q8", "w8a8", "q4"), threads=1):
+    """One bounded sample of the workload through the oracle: each precision
+    x each linear of one block, the whole pipeline on `rows_per_gemm` token
+    rows. The 12 pipelines run on `threads` host threads (the oracle's C
+    calls release the interpreter lock). Returns (gemm ops counted like the
+    GPU arm, wall seconds, threads used)."""
+    jobs = [(name, k, n, fmt) for name, k, n in linears for fmt in fmts]
+    threads = max(1, min(threads, len(jobs)))
+    t0 = time.perf_counter()
+    if threads == 1:
+        res = [_cpu_pipeline(*j, rows_per_gemm, block) for j in jobs]
+    else:
+        with concurrent.futures.ThreadPoolExecutor(threads) as ex:
+            res = list(ex.map(lambda j: _cpu_pipeline(*j, rows_per_gemm, block), jobs))
+    wall = time.perf_counter() - t0
+    return sum(r[0] for r in res), wall, threads
 
 
 def cpu_baseline(rows=16):
-    ops, t = cpu_sample(rows_per_gemm=rows)
-    return {"value": ops / t / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "seconds": t,
-            "sample": f"block 0, all 4 linears x (q8, W8A8, q4): pack + quant + GEMM + epilogue "
-                      f"on {rows} of 432 token rows; single-threaded plain C, fp64 GEMM; "
-                      f"ops counted as 2*rows*N*K per GEMM"}
+    ops1, t1, _ = cpu_sample(rows_per_gemm=rows, threads=1)
+    opsn, tn, nth = cpu_sample(rows_per_gemm=rows, threads=cpu_threads())
+    sample = (f"block 0, all 4 linears x (q8, W8A8, q4): pack + quant + GEMM + epilogue on {rows} "
+              f"of 432 token rows; plain C oracle, fp64 GEMM; ops counted as 2*rows*N*K per GEMM")
+    return {"value": opsn / tn / 1e12, "unit": "TOPS", "cores": nth, "kind": "oracle",
+            "seconds": tn, "sample": sample + f"; the 12 pipelines on {nth} host threads",
+            "single_thread": {"value": ops1 / t1 / 1e12, "cores": 1, "seconds": t1},
+            "host_cores_available": cpu_threads()}
 
 
 def run_reference(args, ws, rank):
     """The oracle as the reference arm, on this arm's metric and workload."""
     if rank != 0:
         return None
+    nth = cpu_threads() if args.ref_threads <= 0 else args.ref_threads
     for _ in range(args.warmup):
-        cpu_sample(rows_per_gemm=1, linears=LINEARS[1:2])
-    ops, t = 0.0, 0.0
+        cpu_sample(rows_per_gemm=1, linears=LINEARS[1:2], fmts=("q8",))
+    ops, t, used = 0.0, 0.0, 1
     rows = max(1, int(args.ref_rows))
     for s in range(args.steps):
-        o, dt = cpu_sample(rows_per_gemm=rows, block=s % BLOCKS)
+        o, dt, used = cpu_sample(rows_per_gemm=rows, block=s % BLOCKS, threads=nth)
         ops += o
         t += dt
     value = ops / t / 1e12
     sample = (f"each step: one block's 4 linears x (q8, W8A8, q4), pack + quant + GEMM + "
-              f"epilogue on {rows} of 432 token rows, single-threaded plain C oracle")
+              f"epilogue on {rows} of 432 token rows, plain C oracle on {used} host threads")
     return {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": WORKLOAD, "tokens": M, "blocks": BLOCKS, "denoise_steps": STEPS,
                        "parallelism": "single process (CPU)"},
-            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": used, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-# ------------------------------------------------------- single-kernel case --
+# ------------------------------------------------------ per-shape cases -----
 
-SWEEP = ([("q8", n, k, m) for m in (1, 16, 432) for _, k, n in synthetic.D1024]
-         + [("w8a8", n, k, m) for m in (432, 4096) for _, k, n in synthetic.D1536]
-         + [("act_quant", 1536, k, m) for m in (432, 4096) for k in (1536, 6144)]
-         + [("q4", n, k, m) for m in (1, 8, 432) for _, k, n in synthetic.D1536]
-         + [("pack_q8", n, k, 1) for _, k, n in synthetic.D1536]
-         + [("pack_q4", n, k, 1) for _, k, n in synthetic.D1536])
+def _d(lin):
+    return {n: (k, nn) for n, k, nn in lin}
 
 
-def run_sweep(args):
-    """Every per-shape case of the q8 (d=1024), W8A8 (d=1536) and q4 (d=1536)
-    workloads, one JSON line each, in one process."""
-    for case, n, k, m in SWEEP:
-        a = argparse.Namespace(**vars(args))
-        a.case, a.shape, a.m = case, f"{n}x{k}", m
-        run_case(a)
-        torch.cuda.empty_cache()
+# (configuration, case, linear name, N, K, M); N, K from the configuration's shapes
+CONFIG_CASES = (
+    [("tiny q8 (256x256, M=64)", "q8", "tiny", 256, 256, 64)]
+    + [("q8 d=1024", "q8", name, n, k, m) for m in (1, 16, 432) for name, k, n in synthetic.D1024]
+    + [("W8A8 d=1536 act quant", "act_quant", "", 0, k, m) for m in (432, 4096) for k in (1536, 6144)]
+    + [("W8A8 d=1536", "w8a8", name, n, k, m) for m in (432, 4096) for name, k, n in synthetic.D1536]
+    + [("q4 d=1536", "q4", name, n, k, m) for m in (1, 8, 432) for name, k, n in synthetic.D1536]
+    + [("fp16 d=1536 (precision ladder)", "f16", name, n, k, m) for m in (1, 432)
+       for name, k, n in synthetic.D1536]
+    + [("pack d=1536", "pack_q8", name, n, k, 0) for name, k, n in synthetic.D1536]
+    + [("pack d=1536", "pack_q4", name, n, k, 0) for name, k, n in synthetic.D1536]
+)
+
+# north_star bars: weight-bound shapes >= 70 % of HBM, large-M W8A8 >= 60 % of int8
+def case_target(case, m):
+    if (case == "q8" and m in (1, 16)) or (case == "q4" and m in (1, 8)):
+        return ("hbm_frac", 0.70)
+    if case == "w8a8" and m == 4096:
+        return ("tensor_frac", 0.60)
+    return None
 
 
-def run_case(args):
-    """One kernel on one shape, launched `reps` times back to back, cycling
-    through enough weight copies to exceed L2 (for ncu captures and per-shape
-    sweeps). Prints one JSON line with the mean launch time."""
+def _case_inputs(case, name, n, k, m):
+    """Seeded inputs of one case (the configuration's own generators)."""
+    if case == "act_quant":
+        return None, synthetic.activation(f"w8a8d1536/act/M{m}/K{k}", m, k, outlier_channel_frac=0.01)
+    if name == "tiny":
+        d = synthetic.tiny_q8()
+        return d["W"], d["X"]
+    if case == "q8":
+        return synthetic.q8_block_d1024(name, m)
+    if case in ("w8a8", "pack_q8"):
+        return synthetic.w8a8_d1536(name, max(m, 1))
+    return synthetic.q4_d1536(name, max(m, 1))
+
+
+def run_case(case, n, k, m, reps=200, name="", R=None, cycle=True):
+    """One kernel on one shape, `reps` launches back to back in one CUDA graph
+    (each launch in stream order after the previous one, as in a layer
+    sequence), cycling through enough copies of what the launch streams --
+    packed weights, or the fp16 weights of a pack, or the activations of the
+    activation quantiser -- to exceed 3x L2. Returns one result dict."""
     import int8_int4_b200 as aq
     dev = torch.device("cuda", torch.cuda.current_device())
-    n, k = (int(v) for v in args.shape.split("x"))
-    m = args.m
-    W = synthetic.weight(f"case/{n}x{k}", n, k).to(dev)
-    X = synthetic.activation(f"case/{m}x{k}", m, k).to(dev)
-    fmt = {"w8a8": "q8", "pack_q8": "q8", "pack_q4": "q4"}.get(args.case, args.case)
-    per_copy = n * k * (2 if args.case.startswith("pack") else (0.5625 if fmt == "q4" else 1))
-    copies = max(1, int(np.ceil(3 * 126e6 / per_copy))) if args.cycle else 1
-    packs = [aq.qpack(fmt, W) for _ in range(1 if args.case.startswith("pack") else copies)]
-    Ws = [W] + [W.clone() for _ in range(copies - 1)] if args.case.startswith("pack") else None
-    Xq = aq.act_quant(X) if args.case == "w8a8" else None
-    Y = torch.empty(m, n, dtype=torch.float16, device=dev)
-
-    def launch(i):
-        if args.case == "act_quant":
-            aq.act_quant(X)
-        elif args.case.startswith("pack"):
-            aq.qpack(fmt, Ws[i % len(Ws)])
-        elif args.case == "w8a8":
-            aq.qgemm("w8a8", Xq[0], *packs[i % copies], sx=Xq[1], out=Y)
+    W, X = _case_inputs(case, name, n, k, m)
+    if case == "act_quant":
+        per_copy = 3 * m * k
+    elif case.startswith("pack"):
+        per_copy = 2 * n * k
+    else:
+        per_copy = {"q8": n * k, "w8a8": n * k, "q4": 0.5625 * n * k, "f16": 2 * n * k}[case]
+    copies = max(1, int(np.ceil(3 * 126e6 / per_copy))) if cycle else 1
+    Y = torch.empty(max(m, 1), max(n, 1), dtype=torch.float16, device=dev)
+    if case == "act_quant":
+        Xs = [X.to(dev) for _ in range(copies)]
+        outs = (torch.empty(m, k, dtype=torch.int8, device=dev), torch.empty(m, dtype=torch.float32, device=dev))
+        launch = lambda i: aq.act_quant(Xs[i % copies], out=outs)
+    elif case.startswith("pack"):
+        fmt = case[5:]
+        Ws = [W.to(dev) for _ in range(copies)]
+        packed = aq.qpack(fmt, Ws[0])
+        launch = lambda i: aq.qpack(fmt, Ws[i % copies], out=packed)
+    else:
+        Wd = W.to(dev)
+        Xd = X.to(dev)
+        if case == "f16":
+            packs = [(Wd.clone(), None) for _ in range(copies)]
         else:
-            aq.qgemm(fmt, X, *packs[i % copies], out=Y)
-
+            p0 = aq.qpack("q8" if case == "w8a8" else case, Wd)
+            packs = [tuple(t.clone() for t in p0) for _ in range(copies)]
+        del Wd
+        kw = {}
+        if case == "w8a8":
+            Xd, kw["sx"] = aq.act_quant(Xd)
+        fmt = case
+        launch = lambda i: aq.qgemm(fmt, Xd, *packs[i % copies], out=Y, **kw)
     for i in range(3):
         launch(i)
     torch.cuda.synchronize()
-    # the reps launches are captured in one CUDA graph, so host launch cost
-    # does not enter the per-kernel time
     s = torch.cuda.Stream()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            for i in range(args.reps):
+            for i in range(reps):
                 launch(i)
     g.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0, e1 = _ev(), _ev()
     e0.record()
     g.replay()
     e1.record()
     torch.cuda.synchronize()
     aq.device_status()
-    us = e0.elapsed_time(e1) * 1e3 / args.reps
-    ops = gemm_ops(m, n, k) if args.case in ("q8", "q4", "w8a8") else 0.0
-    if args.case in ("q8", "q4"):
-        byt = bytes_wo(fmt, m, n, k, False)
-    elif args.case == "w8a8":
-        byt = bytes_w8a8(m, n, k, False)
-    elif args.case == "act_quant":
-        byt = bytes_act_quant(m, k)
+    t = e0.elapsed_time(e1) * 1e-3 / reps
+    del g
+    if case in ("q8", "q4", "w8a8", "f16"):
+        ops = gemm_ops(m, n, k)
+        byt = {"q8": lambda: bytes_wo("q8", m, n, k, False), "q4": lambda: bytes_wo("q4", m, n, k, False),
+               "w8a8": lambda: bytes_w8a8(m, n, k, False), "f16": lambda: bytes_f16(m, n, k, False)}[case]()
+    elif case == "act_quant":
+        ops, byt = 0.0, bytes_act_quant(m, k)
     else:
-        byt = 2 * n * k + (n * k + 4 * n if fmt == "q8" else n * k // 2 + 2 * n * (k // 32))
-    print(json.dumps({"case": args.case, "M": m, "N": n, "K": k, "reps": args.reps,
-                      "weight_copies": copies, "avg_us": us, "tops": ops / us / 1e6,
-                      "gbs": byt / us / 1e3}), flush=True)
+        ops, byt = 0.0, bytes_pack(case[5:], n, k)
+    R = R or roofs(load_peaks()[0])
+    d = {"case": case, "linear": name, "M": m, "N": n, "K": k, "reps": reps, "copies": copies}
+    d.update(roof_entry(ops, byt, t, R["i8"] if case == "w8a8" else R["f16"], R["hbm"]))
+    tgt = case_target(case, m)
+    if tgt:
+        d["target"] = {"of": tgt[0], "frac": tgt[1], "met": d[tgt[0]] >= tgt[1]}
+    return d
+
+
+def run_cases(cases, reps, R):
+    out = []
+    for label, case, name, n, k, m in cases:
+        d = run_case(case, n, k, m, reps=reps, name=name, R=R)
+        d["config"] = label
+        out.append({kk: (round(v, 4) if isinstance(v, float) else v) for kk, v in d.items()})
+        torch.cuda.empty_cache()
+    return out
 
 
 def main(argv=None):
@@ -635,21 +801,28 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--no-fp16", action="store_true", help="skip the fp16 rung of the replay")
     ap.add_argument("--ref-rows", type=int, default=4)
-    ap.add_argument("--case", choices=["q8", "q4", "w8a8", "act_quant", "pack_q8", "pack_q4"],
-                    help="time one kernel on one shape instead of the workload (no JSON bench line)")
-    ap.add_argument("--shape", default="1536x1536", help="NxK of the weight for --case")
+    ap.add_argument("--ref-threads", type=int, default=0, help="reference arm threads (0: all host cores)")
+    ap.add_argument("--case", choices=["q8", "q4", "w8a8", "f16", "act_quant", "pack_q8", "pack_q4"],
+                    help="time one kernel on one shape instead of the workload (no bench line)")
+    ap.add_argument("--shape", default="1536x1536", help="NxK of the weight for --case (K for act_quant)")
     ap.add_argument("--m", type=int, default=432, help="tokens for --case")
     ap.add_argument("--reps", type=int, default=200)
     ap.add_argument("--sweep", action="store_true", help="time every per-shape case (JSON lines)")
     ap.add_argument("--no-cycle", dest="cycle", action="store_false",
-                    help="reuse one weight copy (L2-resident) for --case")
+                    help="reuse one copy (L2-resident) for --case")
     args = ap.parse_args(argv)
     if args.case:
-        run_case(args)
+        dims = [int(v) for v in args.shape.split("x")]
+        n, k = (0, dims[-1]) if args.case == "act_quant" else (dims[0], dims[1])
+        print(json.dumps(run_case(args.case, n, k, args.m, reps=args.reps, cycle=args.cycle)), flush=True)
         return
     if args.sweep:
-        run_sweep(args)
+        R = roofs(load_peaks()[0])
+        for c in CONFIG_CASES:
+            print(json.dumps(run_cases([c], args.reps, R)[0]), flush=True)
         return
     ws, rank, _ = dist_init()
     try:

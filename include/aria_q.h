@@ -9,7 +9,9 @@
  * four precisions -- fp16, q8, W8A8 (8-bit arithmetic on integer tensor
  * cores, the fastest GPU mode) and q4; q8 and W8A8 share one footprint.
  * "Steering is real": a direction vector is added at one transformer block,
- * and alpha = 0 removes it with bit-identical output.
+ * and alpha = 0 removes it with bit-identical output. "Live steering while
+ * streaming": the steering lives inside the captured CUDA graph, so its
+ * strength can change from one step or chunk to the next.
  *
  * Formats (the pages give none; these are the library's fixed readings):
  *   Q8 / W8A8 weights: Wq int8 [N,K] row-major (K contiguous),
@@ -60,7 +62,8 @@ typedef enum {
 typedef enum {
     ARIA_FMT_Q8 = 1,    /* 8-bit weights, fp16 activations (weight-only) */
     ARIA_FMT_Q4 = 2,    /* 4-bit group-32 weights, fp16 activations (weight-only) */
-    ARIA_FMT_W8A8 = 3   /* 8-bit weights (the Q8 pack) x per-token int8 activations */
+    ARIA_FMT_W8A8 = 3,  /* 8-bit weights (the Q8 pack) x per-token int8 activations */
+    ARIA_FMT_F16 = 4    /* unquantised fp16 weights (the fp16 rung of the precision table) */
 } aria_format;
 
 /* Human-readable name of a status code (static string). */
@@ -72,7 +75,8 @@ const char *aria_last_error_message(void);
 /*
  * aria_qpack_size -- bytes of the packed weights and of their scales.
  * ("What aria is": weights packed from fp16 to 8 or 4 bits.)
- *   fmt    ARIA_FMT_Q8 or ARIA_FMT_W8A8 (same pack), or ARIA_FMT_Q4.
+ *   fmt    ARIA_FMT_Q8 or ARIA_FMT_W8A8 (same pack), or ARIA_FMT_Q4. ARIA_FMT_F16
+ *          weights are used unpacked: ARIA_ERR_UNSUPPORTED.
  *   group  0 for Q8 / W8A8 (per output channel); 32 for Q4.
  *   N, K   output and input features of the linear layer (W is [N,K]).
  *   wq_bytes, scale_bytes  host outputs: N*K and 4*N (Q8), N*K/2 and 2*N*K/32 (Q4).
@@ -113,27 +117,34 @@ aria_status aria_act_quant(const void *X, int64_t M, int64_t K, int8_t *Xq, floa
  *   W8A8: main = acc[m,n] * s_x[m] * s_w[n], acc = sum_k Xq*Wq exact int32
  *         (int8 tensor cores); the epilogue is evaluated in fp64 and rounded
  *         once to fp16.
- *   X       device: fp16 [M,K] (Q8, Q4) or int8 [M,K] from aria_act_quant (W8A8).
+ *   F16:  main = sum_k X[m,k] * W[n,k] on the unquantised fp16 weights
+ *         (fp16 tensor cores; "Results": the fp16 column of the table).
+ *   Weight-only and F16 results accumulate in fp32 and are rounded once to fp16.
+ *   X       device: fp16 [M,K] (Q8, Q4, F16) or int8 [M,K] from aria_act_quant (W8A8).
  *   sx      device fp32 [M] (W8A8 only; must be NULL otherwise).
- *   Wq, scales  device, as produced by aria_qpack (W8A8 takes the Q8 pack).
+ *   Wq, scales  device, as produced by aria_qpack (W8A8 takes the Q8 pack);
+ *           F16: Wq is the fp16 weight [N,K] itself and scales must be NULL.
  *   bias    device fp16 [N], or NULL for none.
  *   steer_vec device fp32 [N], or NULL. The steering add ("Steering is real")
  *           is skipped entirely when steer_vec == NULL or alpha == 0, so the
  *           output is then bit-identical to an unsteered call.
  *   Y       device output, fp16 [M,N] row-major. Must not alias any input.
  * Shape rules: M >= 1; N >= 16, N % 16 == 0; K >= 16, K % 16 == 0;
- *   Q4 additionally K % 256 == 0; group as in aria_qpack_size.
+ *   Q4 additionally K % 256 == 0; group as in aria_qpack_size (0 for F16);
+ *   W8A8 additionally K * 127^2 < 2^31 (K <= 133144), so that the exact
+ *   int32 accumulators cannot wrap (ARIA_ERR_UNSUPPORTED otherwise).
  * Deterministic: the same inputs give the same bytes on every call.
  * Stream order: the kernel is launched with programmatic dependent launch,
  *   so it may start while the preceding kernel in `stream` finishes. X, sx,
- *   bias, steer_vec and Y are touched only after that kernel has completed;
- *   the first weight tiles (Wq, and the Q4 scales) are loaded before. Wq and
- *   scales must therefore be complete before the preceding kernel in the
- *   stream starts, or be written by a kernel that does not allow an early
- *   start of its successor (no griddepcontrol.launch_dependents /
- *   cudaTriggerProgrammaticLaunchCompletion before its last write).
- *   aria_qpack's kernels never allow it, so pack-then-GEMM on one stream is
- *   safe.
+ *   bias, steer_vec, a device alpha and Y are touched only after that kernel
+ *   has completed; the first weight tiles (Wq, and the Q4 scales) are loaded
+ *   before. Wq and scales must therefore be complete before the preceding
+ *   kernel in the stream starts, or be written by a kernel that does not
+ *   allow an early start of its successor (no griddepcontrol.launch_dependents
+ *   / cudaTriggerProgrammaticLaunchCompletion before its last write) and
+ *   whose threads make their stores visible at GPU scope and to the async
+ *   proxy before they exit (__threadfence(); fence.proxy.async.global).
+ *   aria_qpack's kernels do both, so pack-then-GEMM on one stream is safe.
  */
 aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
                        const void *X, const float *sx, const void *Wq, const void *scales,
@@ -141,12 +152,34 @@ aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t
                        void *stream);
 
 /*
+ * aria_qgemm_steer_dev -- aria_qgemm with the steering strength read from
+ * device memory when the kernel runs ("Live steering while streaming": the
+ * steering lives inside the captured graph, so control can change
+ * mid-stream; "Run it": the steer spec names a step window, e.g. 0-7).
+ * A CUDA graph captured once can then follow an alpha schedule: capture
+ * step s's steered call with alpha_dev = &schedule[s], and rewrite the
+ * schedule (e.g. with cudaMemcpyAsync) between replays; steps outside the
+ * window hold 0.
+ *   alpha_dev  device fp32 scalar, 4-byte aligned; read after the preceding
+ *              kernel in `stream` has completed. Required when steer_vec is
+ *              not NULL (ARIA_ERR_INVALID_ARG), ignored when it is NULL.
+ *   Every other argument and rule as for aria_qgemm (alpha is *alpha_dev).
+ *   A value of 0 at run time skips the add entirely, so that step's output
+ *   is bit-identical to an unsteered call; a non-zero value gives the same
+ *   bytes as aria_qgemm with that alpha.
+ */
+aria_status aria_qgemm_steer_dev(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
+                                 const void *X, const float *sx, const void *Wq,
+                                 const void *scales, const void *bias, const float *steer_vec,
+                                 const float *alpha_dev, void *Y, void *stream);
+
+/*
  * aria_qgemm_s32 -- the W8A8 integer GEMM alone: C[m,n] = sum_k Xq[m,k]*Wq[n,k]
  * as exact int32 ("Results": 8-bit arithmetic on integer tensor cores). Runs
  * the same tensor-core mainloop as aria_qgemm(ARIA_FMT_W8A8) and stores the
  * raw accumulators, for bit-exact checks.
  *   Xq device int8 [M,K]; Wq device int8 [N,K]; C device output int32 [M,N].
- * Shape rules as for aria_qgemm. The caller keeps K * 127^2 < 2^31.
+ * Shape rules as for aria_qgemm, including K * 127^2 < 2^31 (ARIA_ERR_UNSUPPORTED).
  */
 aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t *Xq, const int8_t *Wq,
                            int32_t *C, void *stream);

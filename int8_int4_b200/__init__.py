@@ -8,12 +8,15 @@ the calls raise.
 
 Method: "A Quantized Native Runtime for On-Device Semantic Audio Generation"
 (aria project page): "What aria is" (weights packed from fp16 to 8 or 4
-bits), "Results" (q8, W8A8 on integer tensor cores, q4), "Steering is real"
-(a direction added at one block, bit-identical at alpha = 0). Formats and
-argument rules are documented in include/aria_q.h.
+bits), "Results" (fp16, q8, W8A8 on integer tensor cores, q4), "Steering is
+real" (a direction added at one block, bit-identical at alpha = 0), "Live
+steering while streaming" (the strength lives inside the captured graph) and
+"Run it" (the steer spec site:block:file:alpha:steps). Formats and argument
+rules are documented in include/aria_q.h.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -25,9 +28,10 @@ LIB_PATH = os.path.join(_PKG, "libaria_q.so")
 ARIA_OK = 0
 STATUS = {0: "ARIA_OK", 1: "ARIA_ERR_INVALID_ARG", 2: "ARIA_ERR_UNSUPPORTED",
           3: "ARIA_ERR_MISALIGNED", 4: "ARIA_ERR_CUDA", 5: "ARIA_ERR_TIMEOUT"}
-FORMATS = {"q8": 1, "q4": 2, "w8a8": 3}
+FORMATS = {"q8": 1, "q4": 2, "w8a8": 3, "f16": 4}
 API = ("aria_status_string", "aria_last_error_message", "aria_qpack_size", "aria_qpack",
-       "aria_act_quant", "aria_qgemm", "aria_qgemm_s32", "aria_device_status")
+       "aria_act_quant", "aria_qgemm", "aria_qgemm_steer_dev", "aria_qgemm_s32",
+       "aria_device_status")
 
 
 class AriaError(RuntimeError):
@@ -55,6 +59,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "aria_qpack": ([I, I, P, I64, I64, P, P, P], I),
         "aria_act_quant": ([P, I64, I64, P, P, P], I),
         "aria_qgemm": ([I, I, I64, I64, I64, P, P, P, P, P, P, ctypes.c_float, P, P], I),
+        "aria_qgemm_steer_dev": ([I, I, I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
         "aria_qgemm_s32": ([I64, I64, I64, P, P, P, P], I),
         "aria_device_status": ([P], I),
     }
@@ -91,6 +96,31 @@ def _dev(t: torch.Tensor | None, name: str, dtype=None):
     return t.data_ptr()
 
 
+def same_device(**tensors):
+    """Every given tensor (None skipped) on one device; returns it. The library
+    launches on the current device and encodes tensor maps from raw pointers,
+    so a tensor on another GPU would be read through the wrong device."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other arguments on {dev}")
+    return dev
+
+
+@contextlib.contextmanager
+def _on(dev):
+    """Make `dev` the current CUDA device for the library call."""
+    if dev is not None and dev.type == "cuda":
+        with torch.cuda.device(dev):
+            yield
+    else:
+        yield
+
+
 def _group(fmt: str, group):
     return (32 if fmt == "q4" else 0) if group is None else int(group)
 
@@ -106,12 +136,14 @@ def _expect(t, name: str, shape, dtype):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
-def check_gemm_args(fmt: str, X, Wq, scales, sx=None, bias=None, steer_vec=None, out=None):
+def check_gemm_args(fmt: str, X, Wq, scales, sx=None, bias=None, steer_vec=None, out=None,
+                    alpha_dev=None):
     """The tensors of one GEMM call agree with each other and with the format
     (include/aria_q.h): X [M,K] (fp16; int8 for W8A8), Wq [N,K] int8 (q8, W8A8)
-    or [N,K/2] uint8 (q4), scales fp32 [N] (q8, W8A8) or fp16 [N,K/32] (q4),
-    sx fp32 [M] (W8A8 only), bias fp16 [N], steer_vec fp32 [N], out fp16 [M,N].
-    Returns (M, N, K)."""
+    or [N,K/2] uint8 (q4) or the fp16 weight [N,K] itself (f16), scales fp32
+    [N] (q8, W8A8) or fp16 [N,K/32] (q4) or None (f16), sx fp32 [M] (W8A8
+    only), bias fp16 [N], steer_vec fp32 [N], alpha_dev one fp32 element,
+    out fp16 [M,N], all on one device. Returns (M, N, K)."""
     if fmt not in FORMATS:
         raise ValueError(f"unknown format {fmt!r}")
     if X.dim() != 2 or Wq.dim() != 2:
@@ -124,6 +156,10 @@ def check_gemm_args(fmt: str, X, Wq, scales, sx=None, bias=None, steer_vec=None,
             raise ValueError("q4 needs K % 32 == 0")
         _expect(Wq, "Wq", (N, K // 2), torch.uint8)
         _expect(scales, "scales", (N, K // 32), torch.float16)
+    elif fmt == "f16":
+        _expect(Wq, "W", (N, K), torch.float16)
+        if scales is not None:
+            raise ValueError("f16 weights take no scales")
     else:
         _expect(Wq, "Wq", (N, K), torch.int8)
         _expect(scales, "scales", (N,), torch.float32)
@@ -135,7 +171,12 @@ def check_gemm_args(fmt: str, X, Wq, scales, sx=None, bias=None, steer_vec=None,
         raise ValueError("sx is for w8a8 only")
     _expect(bias, "bias", (N,), torch.float16)
     _expect(steer_vec, "steer_vec", (N,), torch.float32)
+    if alpha_dev is not None:
+        if alpha_dev.numel() != 1 or alpha_dev.dtype != torch.float32:
+            raise TypeError("alpha_dev must be one float32 element")
     _expect(out, "out", (M, N), torch.float16)
+    same_device(X=X, Wq=Wq, scales=scales, sx=sx, bias=bias, steer_vec=steer_vec, out=out,
+                alpha_dev=alpha_dev)
     return M, N, K
 
 
@@ -146,19 +187,26 @@ def qpack_size(fmt: str, N: int, K: int, group=None):
     return wb.value, sb.value
 
 
-def qpack(fmt: str, W: torch.Tensor, group=None, stream=None):
-    """Pack fp16 W [N,K]: q8/w8a8 -> (int8 [N,K], fp32 [N]); q4 -> (uint8 [N,K/2], fp16 [N,K/32])."""
+def qpack(fmt: str, W: torch.Tensor, group=None, stream=None, out=None):
+    """Pack fp16 W [N,K]: q8/w8a8 -> (int8 [N,K], fp32 [N]); q4 -> (uint8 [N,K/2], fp16 [N,K/32]).
+    ``out`` = (Wq, scales) writes into existing tensors of those shapes."""
     N, K = W.shape
     g = _group(fmt, group)
     qpack_size(fmt, N, K, g)
-    if fmt == "q4":
-        Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=W.device)
-        S = torch.empty(N, K // 32, dtype=torch.float16, device=W.device)
+    q4 = fmt == "q4"
+    shapes = ((N, K // 2), (N, K // 32)) if q4 else ((N, K), (N,))
+    dtypes = (torch.uint8, torch.float16) if q4 else (torch.int8, torch.float32)
+    if out is None:
+        Wq = torch.empty(*shapes[0], dtype=dtypes[0], device=W.device)
+        S = torch.empty(*shapes[1], dtype=dtypes[1], device=W.device)
     else:
-        Wq = torch.empty(N, K, dtype=torch.int8, device=W.device)
-        S = torch.empty(N, dtype=torch.float32, device=W.device)
-    _check(load_library().aria_qpack(FORMATS[fmt], g, _dev(W, "W", torch.float16), N, K,
-                                     Wq.data_ptr(), S.data_ptr(), _stream(stream)))
+        Wq, S = out
+        _expect(Wq, "Wq", shapes[0], dtypes[0])
+        _expect(S, "scales", shapes[1], dtypes[1])
+        same_device(W=W, Wq=Wq, scales=S)
+    with _on(W.device):
+        _check(load_library().aria_qpack(FORMATS[fmt], g, _dev(W, "W", torch.float16), N, K,
+                                         Wq.data_ptr(), S.data_ptr(), _stream(stream)))
     return Wq, S
 
 
@@ -170,23 +218,40 @@ def act_quant(X: torch.Tensor, out=None, stream=None):
         torch.empty(M, dtype=torch.float32, device=X.device))
     _expect(Xq, "Xq", (M, K), torch.int8)
     _expect(sx, "sx", (M,), torch.float32)
-    _check(load_library().aria_act_quant(_dev(X, "X", torch.float16), M, K,
-                                         _dev(Xq, "Xq", torch.int8), _dev(sx, "sx", torch.float32),
-                                         _stream(stream)))
+    dev = same_device(X=X, Xq=Xq, sx=sx)
+    with _on(dev):
+        _check(load_library().aria_act_quant(_dev(X, "X", torch.float16), M, K,
+                                             _dev(Xq, "Xq", torch.int8), _dev(sx, "sx", torch.float32),
+                                             _stream(stream)))
     return Xq, sx
 
 
-def qgemm(fmt: str, X: torch.Tensor, Wq: torch.Tensor, scales: torch.Tensor, sx=None,
-          bias=None, steer_vec=None, alpha: float = 0.0, group=None, out=None, stream=None):
-    """Y [M,N] fp16 = X . dequant(W)^T + bias + alpha*v (see include/aria_q.h)."""
-    M, N, K = check_gemm_args(fmt, X, Wq, scales, sx, bias, steer_vec, out)
+def qgemm(fmt: str, X: torch.Tensor, Wq: torch.Tensor, scales, sx=None,
+          bias=None, steer_vec=None, alpha: float = 0.0, group=None, out=None, stream=None,
+          alpha_dev=None):
+    """Y [M,N] fp16 = X . dequant(W)^T + bias + alpha*v (see include/aria_q.h).
+
+    fmt "f16" takes the fp16 weight [N,K] as Wq and scales=None. With
+    ``alpha_dev`` (one fp32 element on the device, e.g. ``schedule[s:s+1]``)
+    the strength is read from device memory when the kernel runs
+    (aria_qgemm_steer_dev) and ``alpha`` is ignored."""
+    if fmt != "f16" and scales is None:
+        raise ValueError(f"{fmt} needs scales")
+    M, N, K = check_gemm_args(fmt, X, Wq, scales, sx, bias, steer_vec, out, alpha_dev)
     Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=X.device)
     xdt = torch.int8 if fmt == "w8a8" else torch.float16
-    _check(load_library().aria_qgemm(
-        FORMATS[fmt], _group(fmt, group), M, N, K, _dev(X, "X", xdt),
-        _dev(sx, "sx", torch.float32), _dev(Wq, "Wq"), _dev(scales, "scales"),
-        _dev(bias, "bias", torch.float16), _dev(steer_vec, "steer_vec", torch.float32),
-        float(alpha), _dev(Y, "out"), _stream(stream)))
+    lib = load_library()
+    args = (FORMATS[fmt], _group(fmt, group), M, N, K, _dev(X, "X", xdt),
+            _dev(sx, "sx", torch.float32), _dev(Wq, "Wq"), _dev(scales, "scales"),
+            _dev(bias, "bias", torch.float16), _dev(steer_vec, "steer_vec", torch.float32))
+    with _on(X.device):
+        if alpha_dev is not None:
+            if not alpha_dev.is_cuda:
+                raise ValueError("alpha_dev must be a CUDA tensor")
+            _check(lib.aria_qgemm_steer_dev(*args, alpha_dev.data_ptr(), _dev(Y, "out"),
+                                            _stream(stream)))
+        else:
+            _check(lib.aria_qgemm(*args, float(alpha), _dev(Y, "out"), _stream(stream)))
     return Y
 
 
@@ -197,12 +262,56 @@ def qgemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out=None, stream=None):
     _expect(Wq, "Wq", (N, K), torch.int8)
     C = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xq.device)
     _expect(C, "out", (M, N), torch.int32)
-    _check(load_library().aria_qgemm_s32(M, N, K, _dev(Xq, "Xq", torch.int8),
-                                         _dev(Wq, "Wq", torch.int8), _dev(C, "out", torch.int32),
-                                         _stream(stream)))
+    dev = same_device(Xq=Xq, Wq=Wq, out=C)
+    with _on(dev):
+        _check(load_library().aria_qgemm_s32(M, N, K, _dev(Xq, "Xq", torch.int8),
+                                             _dev(Wq, "Wq", torch.int8), _dev(C, "out", torch.int32),
+                                             _stream(stream)))
     return C
 
 
 def device_status(stream=None):
     """Synchronise the stream and raise if a kernel's bounded wait ran out."""
     _check(load_library().aria_device_status(_stream(stream)))
+
+
+# ------------------------------------------------------- steering schedule --
+
+def parse_steer_spec(spec: str) -> dict:
+    """Parse a steer spec ``site:block:file:alpha:steps`` ("Run it", e.g.
+    ``residual:19:directions/small/sour.atns:0.1:0-7``) into its fields.
+    ``steps`` is an inclusive range ``a-b`` or a single step ``a``. The file
+    is only named here: the direction itself is passed to the GEMM as a
+    device vector. Raises ValueError on a malformed spec."""
+    parts = spec.split(":")
+    if len(parts) != 5:
+        raise ValueError(f"steer spec needs 5 fields site:block:file:alpha:steps, got {spec!r}")
+    site, block, path, alpha, steps = parts
+    if not site:
+        raise ValueError("empty steering site")
+    try:
+        block_i = int(block)
+        alpha_f = float(alpha)
+    except ValueError as e:
+        raise ValueError(f"bad block or alpha in {spec!r}") from e
+    if block_i < 0:
+        raise ValueError("block must be >= 0")
+    a, sep, b = steps.partition("-")
+    try:
+        s0 = int(a)
+        s1 = int(b) if sep else s0
+    except ValueError as e:
+        raise ValueError(f"bad step range {steps!r}") from e
+    if s0 < 0 or s1 < s0:
+        raise ValueError(f"bad step range {steps!r}")
+    return {"site": site, "block": block_i, "file": path, "alpha": alpha_f, "steps": (s0, s1)}
+
+
+def steer_schedule(spec, n_steps: int) -> list:
+    """Per-step strengths of a steer spec (a string or parse_steer_spec's
+    dict): alpha inside the inclusive step window, 0.0 outside it (a zero
+    strength skips the add, so those steps are bit-identical to unsteered
+    ones). Feed it to a device tensor read through ``alpha_dev``."""
+    d = parse_steer_spec(spec) if isinstance(spec, str) else spec
+    s0, s1 = d["steps"]
+    return [d["alpha"] if s0 <= s < s1 + 1 else 0.0 for s in range(n_steps)]

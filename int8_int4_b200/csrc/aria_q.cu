@@ -81,19 +81,26 @@ struct DevInfo {
   int smem_optin = 232448;
 };
 
-DevInfo dev_info() {
-  static DevInfo info[16];
-  static bool done[16] = {};
-  static std::mutex mu;
+constexpr int kMaxDevices = 64;
+
+int current_device() {
   int dev = 0;
-  cudaGetDevice(&dev);
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  return dev;
+}
+
+DevInfo dev_info() {
+  static DevInfo info[kMaxDevices];
+  static bool done[kMaxDevices] = {};
+  static std::mutex mu;
+  const int dev = current_device();
   std::lock_guard<std::mutex> g(mu);
-  if (dev >= 0 && dev < 16 && !done[dev]) {
+  if (dev >= 0 && dev < kMaxDevices && !done[dev]) {
     cudaDeviceGetAttribute(&info[dev].sms, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&info[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     done[dev] = true;
   }
-  return (dev >= 0 && dev < 16) ? info[dev] : DevInfo{};
+  return (dev >= 0 && dev < kMaxDevices) ? info[dev] : DevInfo{};
 }
 
 // ----------------------------------------------------------------- GEMM ---
@@ -111,14 +118,14 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  const int unitK = kind == kQ4 ? 256 : 128;
+  const int unitK = kind == kQ4 ? 256 : (kind == kF16 ? 64 : 128);
   p.units = static_cast<int>((K + unitK - 1) / unitK);
 
   // Token tile: up to 256. W8A8 at M <= 512 uses narrower tiles (<= 160):
   // more output tiles fill the SMs, and without a dequant stage the per-tile
   // cost of a narrower MMA is small (measured: 15-25 % faster at M = 432).
   int max_bn = 256;
-  if ((kind == kW8A8 || kind == kS32) && M <= 512) max_bn = 160;
+  if ((kind == kW8A8 || kind == kS32 || kind == kF16) && M <= 512) max_bn = 160;
 #if defined(ARIA_MAX_BN)
   max_bn = ARIA_MAX_BN;  // tuning builds only
 #endif
@@ -231,18 +238,19 @@ void set_pdl(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr) {
   cfg.attrs = attr;
 }
 
-// how many clusters of `size` CTAs of this kernel can be resident at once
-// (cached per size and shared-memory footprint; queried outside any capture
-// on first use)
+// how many clusters of `size` CTAs of this kernel can be resident at once on
+// the current device (cached per device, size and shared-memory footprint;
+// queried outside any capture on first use)
 template <int KIND>
 int max_clusters(int size, int threads, size_t smem) {
   static std::mutex mu;
-  static int cache_size[64], cache_n[64];
+  static int cache_dev[64], cache_size[64], cache_n[64];
   static size_t cache_smem[64];
   static int used = 0;
+  const int dev = current_device();
   std::lock_guard<std::mutex> g(mu);
   for (int i = 0; i < used; ++i)
-    if (cache_size[i] == size && cache_smem[i] == smem) return cache_n[i];
+    if (cache_dev[i] == dev && cache_size[i] == size && cache_smem[i] == smem) return cache_n[i];
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(size, 1, 1);
   cfg.blockDim = dim3(threads, 1, 1);
@@ -260,6 +268,7 @@ int max_clusters(int size, int threads, size_t smem) {
     n = 0;
   }
   if (used < 64) {
+    cache_dev[used] = dev;
     cache_size[used] = size;
     cache_smem[used] = smem;
     cache_n[used] = n;
@@ -268,17 +277,29 @@ int max_clusters(int size, int threads, size_t smem) {
   return n;
 }
 
+// Raise a kernel's dynamic shared-memory limit to the device's opt-in
+// maximum, once per kernel and device (the attribute is per device).
+template <typename F>
+aria_status opt_in_smem(F* kfn, bool (&done)[kMaxDevices], std::mutex& mu) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return fail(ARIA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> g(mu);
+  if (done[dev]) return ARIA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       dev_info().smem_optin);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done[dev] = true;
+  return ARIA_OK;
+}
+
 template <int KIND>
 aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap& ts,
                         const CUtensorMap& tx, cudaStream_t st) {
   auto kfn = aria::qgemm_kernel<KIND>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    dev_info().smem_optin);
-  });
-  if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute");
+  static bool attr_done[kMaxDevices] = {};
+  static std::mutex attr_mu;
+  aria_status as = opt_in_smem(kfn, attr_done, attr_mu);
+  if (as != ARIA_OK) return as;
   aria::GemmParams prm = pl.p;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
@@ -342,6 +363,8 @@ ARIA_API aria_status aria_qpack_size(aria_format fmt, int group, int64_t N, int6
     *scale_bytes = static_cast<size_t>(N) * 4;
     return ARIA_OK;
   }
+  if (fmt == ARIA_FMT_F16)
+    return fail(ARIA_ERR_UNSUPPORTED, "fp16 weights are used as they are, not packed");
   if (fmt == ARIA_FMT_Q4) {
     if (group != 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 supports group = 32 only");
     if (K % 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 needs K % 32 == 0");
@@ -407,12 +430,16 @@ ARIA_API aria_status aria_act_quant(const void* X, int64_t M, int64_t K, int8_t*
 
 static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const void* X,
                               const float* sx, const void* Wq, const void* scales,
-                              const void* bias, const float* steer, float alpha, void* Y,
-                              cudaStream_t st) {
+                              const void* bias, const float* steer, float alpha,
+                              const float* alpha_dev, void* Y, cudaStream_t st) {
   using namespace aria;
   aria_status s = check_gemm_shape(M, N, K);
   if (s != ARIA_OK) return s;
   if (kind == kQ4 && K % 256) return fail(ARIA_ERR_UNSUPPORTED, "q4 GEMM needs K % 256 == 0");
+  // exact int32 accumulation: |acc| <= K * 127^2 must stay below 2^31
+  if ((kind == kW8A8 || kind == kS32) && K * 127 * 127 > INT32_MAX)
+    return fail(ARIA_ERR_UNSUPPORTED, "int8 GEMM needs K * 127^2 < 2^31 (K <= %lld), got K=%lld",
+                (long long)(INT32_MAX / (127 * 127)), (long long)K);
   Plan pl;
   if ((s = plan_gemm(kind, M, N, K, &pl)) != ARIA_OK) return s;
   CUtensorMap tw, ts, tx;
@@ -423,54 +450,93 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
     if ((s = make_map(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, N, K / 32, 8, 128,
                       CU_TENSOR_MAP_SWIZZLE_NONE)) != ARIA_OK) return s;
+  } else if (kind == kF16) {
+    if ((s = make_map(&tw, Wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, K, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   } else {
     if ((s = make_map(&tw, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, 128, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   }
-  if (kind == kQ8 || kind == kQ4) {
+  if (kind == kQ8 || kind == kQ4 || kind == kF16) {
     if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, 64, bn,
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   } else {
     if ((s = make_map(&tx, X, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, 128, bn,
                       CU_TENSOR_MAP_SWIZZLE_128B)) != ARIA_OK) return s;
   }
-  pl.p.sw = static_cast<const float*>(kind == kQ4 ? nullptr : scales);
+  pl.p.sw = static_cast<const float*>((kind == kQ4 || kind == kF16) ? nullptr : scales);
   pl.p.sx = sx;
   pl.p.bias = static_cast<const __half*>(bias);
-  pl.p.steer = (steer && alpha != 0.0f) ? steer : nullptr;  // skip, not "+ 0*v"
-  pl.p.alpha = alpha;
+  // skip, not "+ 0*v": a host alpha of 0 drops the vector here; a device
+  // alpha is tested in the kernel
+  pl.p.steer = (steer && (alpha_dev || alpha != 0.0f)) ? steer : nullptr;
+  pl.p.alpha = pl.p.steer ? alpha : 0.0f;
+  pl.p.alpha_dev = pl.p.steer ? alpha_dev : nullptr;
   pl.p.Y = Y;
-  if (!pl.p.steer) pl.p.alpha = 0.0f;
   switch (kind) {
     case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, st);
     case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, st);
     case kW8A8: return launch_gemm<kW8A8>(pl, tw, tw, tx, st);
     case kS32: return launch_gemm<kS32>(pl, tw, tw, tx, st);
+    case kF16: return launch_gemm<kF16>(pl, tw, tw, tx, st);
   }
   return fail(ARIA_ERR_INVALID_ARG, "unknown kind");
+}
+
+// argument checks shared by aria_qgemm and aria_qgemm_steer_dev; sets *kind
+static aria_status check_qgemm_args(aria_format fmt, int group, const void* X, const float* sx,
+                                    const void* Wq, const void* scales, const void* bias,
+                                    const float* steer_vec, const void* Y, int* kind) {
+  if (!X || !Wq || !Y) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  if (fmt == ARIA_FMT_Q8 || fmt == ARIA_FMT_W8A8) {
+    if (group != 0) return fail(ARIA_ERR_UNSUPPORTED, "q8 scales are per output channel: group must be 0");
+    *kind = fmt == ARIA_FMT_Q8 ? aria::kQ8 : aria::kW8A8;
+  } else if (fmt == ARIA_FMT_Q4) {
+    if (group != 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 supports group = 32 only");
+    *kind = aria::kQ4;
+  } else if (fmt == ARIA_FMT_F16) {
+    if (group != 0) return fail(ARIA_ERR_UNSUPPORTED, "fp16 weights have no groups: group must be 0");
+    *kind = aria::kF16;
+  } else {
+    return fail(ARIA_ERR_INVALID_ARG, "unknown format %d", (int)fmt);
+  }
+  if (*kind == aria::kF16) {
+    if (scales) return fail(ARIA_ERR_INVALID_ARG, "fp16 weights take no scales (pass NULL)");
+  } else if (!scales) {
+    return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  }
+  if (*kind == aria::kW8A8 && !sx) return fail(ARIA_ERR_INVALID_ARG, "W8A8 needs sx");
+  if (*kind != aria::kW8A8 && sx) return fail(ARIA_ERR_INVALID_ARG, "sx is for W8A8 only");
+  for (const void* q : {X, static_cast<const void*>(sx), Wq, scales, bias,
+                        static_cast<const void*>(steer_vec), Y})
+    if (q && !aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  return ARIA_OK;
 }
 
 ARIA_API aria_status aria_qgemm(aria_format fmt, int group, int64_t M, int64_t N, int64_t K,
                                 const void* X, const float* sx, const void* Wq, const void* scales,
                                 const void* bias, const float* steer_vec, float alpha, void* Y,
                                 void* stream) {
-  if (!X || !Wq || !scales || !Y) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
   int kind = 0;
-  if (fmt == ARIA_FMT_Q8 || fmt == ARIA_FMT_W8A8) {
-    if (group != 0) return fail(ARIA_ERR_UNSUPPORTED, "q8 scales are per output channel: group must be 0");
-    kind = fmt == ARIA_FMT_Q8 ? aria::kQ8 : aria::kW8A8;
-  } else if (fmt == ARIA_FMT_Q4) {
-    if (group != 32) return fail(ARIA_ERR_UNSUPPORTED, "q4 supports group = 32 only");
-    kind = aria::kQ4;
-  } else {
-    return fail(ARIA_ERR_INVALID_ARG, "unknown format %d", (int)fmt);
-  }
-  if (kind == aria::kW8A8 && !sx) return fail(ARIA_ERR_INVALID_ARG, "W8A8 needs sx");
-  if (kind != aria::kW8A8 && sx) return fail(ARIA_ERR_INVALID_ARG, "sx is for W8A8 only");
-  for (const void* q : {X, static_cast<const void*>(sx), Wq, scales, bias,
-                        static_cast<const void*>(steer_vec), static_cast<const void*>(Y)})
-    if (q && !aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
-  return qgemm_impl(kind, M, N, K, X, sx, Wq, scales, bias, steer_vec, alpha, Y,
+  aria_status s = check_qgemm_args(fmt, group, X, sx, Wq, scales, bias, steer_vec, Y, &kind);
+  if (s != ARIA_OK) return s;
+  return qgemm_impl(kind, M, N, K, X, sx, Wq, scales, bias, steer_vec, alpha, nullptr, Y,
+                    static_cast<cudaStream_t>(stream));
+}
+
+ARIA_API aria_status aria_qgemm_steer_dev(aria_format fmt, int group, int64_t M, int64_t N,
+                                          int64_t K, const void* X, const float* sx,
+                                          const void* Wq, const void* scales, const void* bias,
+                                          const float* steer_vec, const float* alpha_dev, void* Y,
+                                          void* stream) {
+  int kind = 0;
+  aria_status s = check_qgemm_args(fmt, group, X, sx, Wq, scales, bias, steer_vec, Y, &kind);
+  if (s != ARIA_OK) return s;
+  if (steer_vec && !alpha_dev)
+    return fail(ARIA_ERR_INVALID_ARG, "a steering vector needs a device alpha");
+  if (alpha_dev && (reinterpret_cast<uintptr_t>(alpha_dev) & 3u))
+    return fail(ARIA_ERR_MISALIGNED, "alpha_dev must be 4-byte aligned");
+  return qgemm_impl(kind, M, N, K, X, sx, Wq, scales, bias, steer_vec, 0.0f, alpha_dev, Y,
                     static_cast<cudaStream_t>(stream));
 }
 
@@ -479,7 +545,7 @@ ARIA_API aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_
   if (!Xq || !Wq || !C) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
   if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(C))
     return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
-  return qgemm_impl(aria::kS32, M, N, K, Xq, nullptr, Wq, Wq, nullptr, nullptr, 0.0f, C,
+  return qgemm_impl(aria::kS32, M, N, K, Xq, nullptr, Wq, Wq, nullptr, nullptr, 0.0f, nullptr, C,
                     static_cast<cudaStream_t>(stream));
 }
 

@@ -1,8 +1,10 @@
 // qgemm.cuh -- quantized GEMMs on the 5th-generation tensor cores (tcgen05).
 //
-// "Results" (aria project page): the transformer runs at q8 or q4 weight-only
-// precision, or as W8A8 with 8-bit arithmetic on integer tensor cores; the
-// steering direction ("Steering is real") is added to one block's output.
+// "Results" (aria project page): the transformer runs at fp16, at q8 or q4
+// weight-only precision, or as W8A8 with 8-bit arithmetic on integer tensor
+// cores; the steering direction ("Steering is real") is added to one block's
+// output, with a strength that may live in device memory so that a captured
+// graph follows a schedule ("Live steering while streaming").
 //
 // One kernel template serves all formats. Orientation is swapped: the MMA's
 // 128-row A operand is a tile of 128 output channels (weight rows) and the
@@ -15,7 +17,7 @@
 // (TMA by lane 0, tcgen05.mma / commit by elect.sync), which keeps the issue
 // loops on the uniform datapath.
 //   warp 0       TMA producer of weight tiles (raw packed bytes for q8/q4; for
-//                W8A8 the int8 weight and activation tiles of each stage). The
+//                W8A8 and fp16 the weight and activation tiles of each stage). The
 //                first ring of weight tiles is loaded before the wait on the
 //                preceding kernel (programmatic dependent launch).
 //   warp 1       TMEM allocator (two accumulator buffers) and MMA issuer
@@ -23,7 +25,7 @@
 //   warps 4..7   epilogue: TMEM -> registers -> scale, bias, steer -> fp16 ->
 //                transposed through shared memory -> coalesced 16-byte stores;
 //                overlaps the next tile's mainloop through the second
-//                accumulator buffer (W8A8 uses warps 8..11 for it as well)
+//                accumulator buffer (W8A8 and fp16 use warps 8..11 for it as well)
 //   warps 8..11  q8/q4: dequantise raw weights into fp16 A tiles (one weight
 //                row per thread; exact int8 -> fp16; fp16 code*scale for q4);
 //                they take part in the epilogue of the CTA's last tile
@@ -41,7 +43,7 @@
 
 namespace aria {
 
-enum GemmKind : int { kQ8 = 1, kQ4 = 2, kW8A8 = 3, kS32 = 4 };
+enum GemmKind : int { kQ8 = 1, kQ4 = 2, kW8A8 = 3, kS32 = 4, kF16 = 5 };
 
 constexpr int kTileN = 128;              // weight rows per tile (MMA M)
 constexpr uint32_t kATile = 16384;       // 128 rows x 128 bytes
@@ -53,7 +55,7 @@ constexpr int kL2Ahead = 4;              // weight units prefetched into L2 ahea
 struct GemmParams {
   int M, N, K;
   int BN;                 // tokens per tile (MMA N): multiple of 16, <= 256
-  int units;              // K units: 128 (q8, W8A8) or 256 (q4) elements
+  int units;              // K units: 128 (q8, W8A8), 256 (q4) or 64 (fp16) elements
   int splits;             // CTAs per cluster along K (1 = persistent over tiles)
   int tiles_n, tiles;     // weight-row tiles, total output tiles
   int n_raw, n_a, n_x;    // ring depths (raw packed weights; stages of A + X; n_x == n_a)
@@ -62,19 +64,23 @@ struct GemmParams {
   const float* sw;        // per-channel weight scale (q8, W8A8)
   const float* sx;        // per-token activation scale (W8A8)
   const __half* bias;     // [N] or null
-  const float* steer;     // [N] or null (null also when alpha == 0)
+  const float* steer;     // [N] or null (null also when a host alpha is 0)
   float alpha;
+  const float* alpha_dev; // device alpha, read after the dependency wait; null: use `alpha`
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
 template <int KIND>
 struct KindTraits {
   static constexpr bool kDequant = (KIND == kQ8 || KIND == kQ4);
-  static constexpr bool kF16 = kDequant;                    // MMA kind::f16 vs kind::i8
+  static constexpr bool kMmaF16 = kDequant || KIND == kF16; // MMA kind::f16 vs kind::i8
   static constexpr int kKbPerUnit = KIND == kQ8 ? 2 : (KIND == kQ4 ? 4 : 1);
-  static constexpr int kXElemsPerKb = kF16 ? 64 : 128;      // 128 bytes of K per row
+  static constexpr int kXElemsPerKb = kMmaF16 ? 64 : 128;   // 128 bytes of K per row
+  // x coordinate step of one K unit in the weight tensor map: 128 bytes of
+  // packed weights (q8, q4, W8A8) or 64 fp16 weights (fp16)
+  static constexpr int kWUnitX = KIND == kF16 ? 64 : 128;
   static constexpr int kThreads = 384;
-  static constexpr int kEpiWarps = kDequant ? 4 : 8;   // W8A8 / S32 use warps 8..11 for the epilogue too
+  static constexpr int kEpiWarps = kDequant ? 4 : 8;   // W8A8 / S32 / fp16 use warps 8..11 for the epilogue too
   static constexpr uint32_t kOutBytes = KIND == kS32 ? 4 : 2;
   static constexpr uint32_t kStageBuf = kEpiRows * 32 * kOutBytes;  // one warp's store box
 };
@@ -130,19 +136,28 @@ struct RowConst {
   bool has_bias = false, has_steer = false;
 };
 
+// The steering strength of this launch: the host value, or the device value
+// (read after the dependency wait, so a preceding kernel may have written
+// it). A zero strength skips the add entirely, which keeps the output
+// bit-identical to an unsteered call.
+__device__ __forceinline__ float steer_alpha(const GemmParams& p) {
+  return p.alpha_dev ? *p.alpha_dev : p.alpha;
+}
+
 template <int KIND>
 __device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) {
   RowConst<KIND> c;
   if (n >= p.N) return c;
   c.has_bias = p.bias != nullptr;
-  c.has_steer = p.steer != nullptr;
+  const float alpha = p.steer ? steer_alpha(p) : 0.0f;
+  c.has_steer = p.steer != nullptr && alpha != 0.0f;
   if constexpr (KIND == kW8A8) {
     c.sw = __ldg(p.sw + n);
     c.sw_up = __fmul_rn(c.sw, 1.0f + 0x1p-21f);
     c.sw_dn = __fmul_rn(c.sw, 1.0f - 0x1p-21f);
     if (c.has_bias) c.bias = __half2float(p.bias[n]);
     if (c.has_steer) {
-      c.alpha = p.alpha;
+      c.alpha = alpha;
       c.v = __ldg(p.steer + n);
       c.av_hi = __fmul_rn(c.alpha, c.v);
       c.av_lo = __fmaf_rn(c.alpha, c.v, -c.av_hi);  // exact remainder of the product
@@ -151,7 +166,7 @@ __device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) 
     if constexpr (KIND == kQ8) c.sw = __ldg(p.sw + n);
     if (c.has_bias) c.bias = __half2float(p.bias[n]);
     if (c.has_steer) {
-      c.alpha = p.alpha;
+      c.alpha = alpha;
       c.v = __ldg(p.steer + n);
     }
   }
@@ -232,6 +247,15 @@ __device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float
     return epi_w8a8_fp64(acc, sx, sw, bias, alpha, v, has_bias, has_steer);
   // midpoint case: |yh| exactly halfway between |h| and its neighbour
   const float ay = fabsf(yh);
+  const float yl_away = yh < 0.0f ? -yl : yl;       // yl measured away from zero
+  if (ay == 65520.0f) {
+    // the midpoint between the largest finite value and overflow: the
+    // conversion ties up to infinity, but a value just below it (yl pointing
+    // toward zero) rounds to the largest finite magnitude 65504
+    if (yl_away < 0.0f)
+      return __ushort_as_half(static_cast<unsigned short>((__half_as_ushort(h) & 0x8000u) | 0x7BFFu));
+    return h;
+  }
   const float ar = fabsf(__half2float(h));
   const float d = __fsub_rn(ay, ar);                // exact (Sterbenz, or ar == 0)
   if (d != 0.0f && ar < 65504.0f) {
@@ -247,8 +271,7 @@ __device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float
     if (fabsf(d) == half_gap) {
       // yh on the midpoint: yl != 0 decides the side; with yl == 0 the value
       // is the midpoint itself and the conversion's tie-to-even stands
-      const float yl_mag = yh < 0.0f ? -yl : yl;    // yl measured away from zero
-      if (yl_mag != 0.0f && (yl_mag > 0.0f) == (d > 0.0f)) {
+      if (yl_away != 0.0f && (yl_away > 0.0f) == (d > 0.0f)) {
         const uint32_t nb = d > 0.0f ? hb + 1u : hb - 1u;
         h = __ushort_as_half(static_cast<unsigned short>((__half_as_ushort(h) & 0x8000u) | nb));
       }
@@ -286,7 +309,8 @@ __device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst
   return w8a8_fixup(h, acc, sx, c.sw, c.bias, c.alpha, c.v, c.has_bias, c.has_steer, v.yh, v.yl);
 }
 
-// q8 / q4: fp32, (acc * s_w) + bias, then + alpha*v[n] (one fma), one rounding to fp16
+// q8 / q4 / fp16: fp32, (acc * s_w) (q8 only) + bias, then + alpha*v[n] (one
+// fma), one rounding to fp16
 template <int KIND>
 __device__ __forceinline__ __half epi_wo(float acc, const RowConst<KIND>& c) {
   float y = acc;
@@ -525,14 +549,14 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       if (lane == 0) {
         for (int i = 0; i < pre; ++i) {
           mbar_arrive_expect_tx(st_full + i, kATile + p.x_stage);
-          tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * 128, n0, pol);
+          tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * T::kWUnitX, n0, pol);
         }
       }
     }
     issued_w = pre;
     if (lane == 0) {  // and the next units into L2
       for (int i = pre; i < nu && i < pre + kL2Ahead; ++i) {
-        tma_prefetch_2d(&tmW, (u_begin + i) * 128, n0);
+        tma_prefetch_2d(&tmW, (u_begin + i) * T::kWUnitX, n0);
         if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
       }
     }
@@ -589,16 +613,18 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             // the weight half went out before the dependency wait (the barrier
             // already expects both halves): add the activation half
             if (lane == 0)
-              tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * 128, m0, polx);
+              tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * T::kXElemsPerKb, m0,
+                          polx);
             if (++s == p.n_a) { s = 0; ph ^= 1u; }
             continue;
           }
           if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2))) break;
           if (lane == 0) {
-            if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * 128, n0);
+            if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * T::kWUnitX, n0);
             mbar_arrive_expect_tx(st_full + s, kATile + p.x_stage);
-            tma_load_2d(&tmW, st_full + s, abuf + s * kATile, (u_begin + kb) * 128, n0, pol);
-            tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * 128, m0, polx);
+            tma_load_2d(&tmW, st_full + s, abuf + s * kATile, (u_begin + kb) * T::kWUnitX, n0, pol);
+            tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * T::kXElemsPerKb, m0,
+                        polx);
           }
           ++issued_w;
           if (++s == p.n_a) { s = 0; ph ^= 1u; }
@@ -626,7 +652,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    const uint32_t idesc = T::kF16 ? idesc_f16_f32(p.BN) : idesc_s8_s32(p.BN);
+    const uint32_t idesc = T::kMmaF16 ? idesc_f16_f32(p.BN) : idesc_s8_s32(p.BN);
     int ti = 0, sa = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -644,7 +670,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sa * p.x_stage));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
-          if constexpr (T::kF16)
+          if constexpr (T::kMmaF16)
             umma_f16_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
           else
             umma_i8_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);

@@ -46,13 +46,22 @@ __device__ __forceinline__ uint2 quant8_i8(const uint4& v, float s, bool zero) {
   return make_uint2(w[0], w[1]);
 }
 
+// A GEMM loads its first packed weight tiles (with TMA, the async proxy)
+// before it waits for the preceding kernel. A pack kernel therefore never
+// lets its successor start early, and every thread ends with its stores
+// ordered at GPU scope and toward the async proxy, so that the pack's
+// completion implies that a following GEMM's tile loads see the bytes.
+__device__ __forceinline__ void publish_packed_stores() {
+  __threadfence();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // One CTA per row: s[r] = absmax / 127, q = clamp(rhe(x / s), -127, 127).
 // Row r of X starts 16-byte aligned (K % 8 == 0); the first kRowCached
 // chunks of each thread stay in registers between the two passes.
 // `early_dependents`: let the next kernel in the stream start its set-up
-// now (activation quantisation). Weight packing passes false: a GEMM reads
-// packed weights before it waits for the preceding kernel, so it must not
-// start before the pack has finished.
+// now (activation quantisation). Weight packing passes false and publishes
+// its stores (see publish_packed_stores).
 __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half* __restrict__ X,
                                                                    int K, int8_t* __restrict__ Q,
                                                                    float* __restrict__ S,
@@ -96,14 +105,15 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half*
   }
   for (int c = threadIdx.x + kRowCached * kRowThreads; c < nchunk; c += kRowThreads)
     qr[c] = quant8_i8(__ldg(xr + c), s, zero);
+  if (!early_dependents) publish_packed_stores();
 }
 
 // q4 pack: one thread per 16-byte chunk (8 consecutive k of one row); four
 // consecutive lanes form a group of 32 and share its absmax by shuffles.
 // s16 = fp16_rn(absmax / 7); code = clamp(rhe(w / float(s16)), -7, 7) + 8,
 // even k in the low nibble. Loop bounds are warp-uniform so every lane
-// takes part in the shuffles. No early start of the next kernel: a GEMM
-// reads packed weights before it waits for the preceding kernel.
+// takes part in the shuffles. No early start of the next kernel, and the
+// stores are published before the threads exit (see publish_packed_stores).
 __global__ void __launch_bounds__(256) pack_q4_kernel(const __half* __restrict__ W,
                                                       int64_t nchunk,
                                                       uint32_t* __restrict__ P,
@@ -135,6 +145,7 @@ __global__ void __launch_bounds__(256) pack_q4_kernel(const __half* __restrict__
       if ((c & 3) == 0) S[c >> 2] = s16;
     }
   }
+  publish_packed_stores();
 }
 
 }  // namespace aria

@@ -181,3 +181,107 @@ def test_binding_rejects_inconsistent_arguments(fmt, field, bad):
         a[field] = torch.zeros(8, dtype=torch.float32)
     with pytest.raises((ValueError, TypeError)):
         aq.check_gemm_args(fmt, **a)
+
+
+# ---------------------------------------------------- later argument rules --
+
+KMAX_I8 = (2 ** 31 - 1) // (127 * 127)       # 133144: largest K whose |acc| <= K*127^2 fits int32
+
+
+def test_int8_gemm_rejects_k_that_could_wrap_int32(lib):
+    k_bad = (KMAX_I8 // 16 + 1) * 16             # the first multiple of 16 above the limit
+    assert k_bad * 127 * 127 > 2 ** 31 - 1
+    assert lib.aria_qgemm(3, 0, 4, 16, k_bad, OK_PTR, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0,
+                          OK_PTR, None) == 2
+    assert b"K" in lib.aria_last_error_message()
+    assert lib.aria_qgemm_s32(4, 16, k_bad, OK_PTR, OK_PTR, OK_PTR, None) == 2
+
+
+def test_f16_format_rules(lib):
+    # fp16 weights are used as they are: no pack, no scales, no groups
+    with pytest.raises(aq.AriaError) as e:
+        aq.qpack_size("f16", 16, 16)
+    assert e.value.status == 2
+    assert lib.aria_qpack(4, 0, OK_PTR, 16, 16, OK_PTR, OK_PTR, None) == 2
+    assert lib.aria_qgemm(4, 0, 4, 16, 16, OK_PTR, None, OK_PTR, OK_PTR, None, None, 0.0, OK_PTR,
+                          None) == 1                                        # scales given
+    assert lib.aria_qgemm(4, 32, 4, 16, 16, OK_PTR, None, OK_PTR, None, None, None, 0.0, OK_PTR,
+                          None) == 2                                        # a group
+    assert lib.aria_qgemm(4, 0, 4, 16, 16, OK_PTR, OK_PTR, OK_PTR, None, None, None, 0.0, OK_PTR,
+                          None) == 1                                        # sx
+    assert lib.aria_qgemm(4, 0, 4, 24, 16, OK_PTR, None, OK_PTR, None, None, None, 0.0, OK_PTR,
+                          None) == 2                                        # N % 16
+
+
+def test_device_alpha_rules(lib):
+    P = ctypes.c_void_p
+    # a steering vector without a device alpha
+    assert lib.aria_qgemm_steer_dev(1, 0, 4, 16, 16, OK_PTR, None, OK_PTR, OK_PTR, None, OK_PTR,
+                                    None, OK_PTR, None) == 1
+    # alpha is one fp32 value: 4-byte alignment is required, 16 is not
+    assert lib.aria_qgemm_steer_dev(1, 0, 4, 16, 16, OK_PTR, None, OK_PTR, OK_PTR, None, OK_PTR,
+                                    P(0x10002), OK_PTR, None) == 3
+    # the aria_qgemm rules apply unchanged
+    assert lib.aria_qgemm_steer_dev(3, 0, 4, 16, 16, OK_PTR, None, OK_PTR, OK_PTR, None, OK_PTR,
+                                    P(0x10004), OK_PTR, None) == 1         # W8A8 without sx
+    assert lib.aria_qgemm_steer_dev(1, 0, 4, 24, 16, OK_PTR, None, OK_PTR, OK_PTR, None, OK_PTR,
+                                    P(0x10004), OK_PTR, None) == 2         # N % 16
+
+
+def test_binding_f16_arguments():
+    import torch
+    M, N, K = 8, 32, 64
+    X = torch.zeros(M, K, dtype=torch.float16)
+    W = torch.zeros(N, K, dtype=torch.float16)
+    assert aq.check_gemm_args("f16", X, W, None) == (M, N, K)
+    with pytest.raises(ValueError):
+        aq.check_gemm_args("f16", X, W, torch.zeros(N, dtype=torch.float32))
+    with pytest.raises(TypeError):
+        aq.check_gemm_args("f16", X, W.to(torch.int8), None)
+
+
+def test_binding_rejects_tensors_on_different_devices():
+    """The library launches on one device and reads raw pointers: a tensor
+    on another device must be refused before any call."""
+    import torch
+    a = _args("q8")
+    a["out"] = torch.zeros(8, 32, dtype=torch.float16, device="meta")
+    with pytest.raises(ValueError, match="out"):
+        aq.check_gemm_args("q8", **a)
+    with pytest.raises(ValueError):
+        aq.same_device(X=torch.zeros(2), Y=torch.zeros(2, device="meta"))
+    assert aq.same_device(X=torch.zeros(2), Y=None, Z=torch.zeros(3)) == torch.device("cpu")
+
+
+def test_binding_alpha_dev_must_be_one_float():
+    import torch
+    a = _args("q8")
+    with pytest.raises(TypeError):
+        aq.check_gemm_args("q8", **a, alpha_dev=torch.zeros(2, dtype=torch.float32))
+    with pytest.raises(TypeError):
+        aq.check_gemm_args("q8", **a, alpha_dev=torch.zeros(1, dtype=torch.float16))
+    assert aq.check_gemm_args("q8", **a, alpha_dev=torch.zeros(1, dtype=torch.float32)) == (8, 32, 256)
+
+
+# --------------------------------------------- steer spec and step window --
+# "Run it" (aria project page): --steer residual:19:directions/small/sour.atns:0.1:0-7
+
+def test_parse_steer_spec_of_the_pages():
+    d = aq.parse_steer_spec("residual:19:directions/small/sour.atns:0.1:0-7")
+    assert d == {"site": "residual", "block": 19, "file": "directions/small/sour.atns",
+                 "alpha": 0.1, "steps": (0, 7)}
+    assert aq.parse_steer_spec("residual:12:v.npy:0.3:4")["steps"] == (4, 4)
+
+
+@pytest.mark.parametrize("spec", ["residual:19:f:0.1", "residual:x:f:0.1:0-7", "residual:19:f:a:0-7",
+                                  "residual:19:f:0.1:5-2", "residual:-1:f:0.1:0-7", ":19:f:0.1:0-7",
+                                  "residual:19:f:0.1:0-"])
+def test_parse_steer_spec_rejects_malformed(spec):
+    with pytest.raises(ValueError):
+        aq.parse_steer_spec(spec)
+
+
+def test_steer_schedule_window():
+    assert aq.steer_schedule("residual:12:v:0.3:0-7", 8) == [0.3] * 8
+    assert aq.steer_schedule("residual:12:v:0.5:2-4", 8) == [0, 0, 0.5, 0.5, 0.5, 0, 0, 0]
+    assert aq.steer_schedule("residual:12:v:0.5:6-9", 8) == [0] * 6 + [0.5, 0.5]   # clipped to the run

@@ -79,3 +79,54 @@ def test_peaks_measured_or_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))   # no MEASURED_PEAKS.json there
     peaks, src = bench.load_peaks()
     assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+
+
+def test_per_config_cases_cover_every_configured_shape():
+    """Every per-shape case of the benchmark configurations is timed: the tiny
+    q8 case, q8 d=1024 at M in {1,16,432}, W8A8 d=1536 at M in {432,4096}
+    with its activation quantisation, q4 d=1536 at M in {1,8,432}, plus the
+    fp16 rung and the two packs."""
+    cases = {(c, n, k, m) for _, c, _, n, k, m in bench.CONFIG_CASES}
+    for _, k, n in synthetic.D1024:
+        for m in (1, 16, 432):
+            assert ("q8", n, k, m) in cases
+    for _, k, n in synthetic.D1536:
+        for m in (432, 4096):
+            assert ("w8a8", n, k, m) in cases
+        for m in (1, 8, 432):
+            assert ("q4", n, k, m) in cases
+        assert ("pack_q8", n, k, 0) in cases and ("pack_q4", n, k, 0) in cases
+    for m in (432, 4096):
+        for k in (1536, 6144):
+            assert ("act_quant", 0, k, m) in cases
+    assert ("q8", 256, 256, 64) in cases
+    assert len(bench.CONFIG_CASES) == len(cases)          # no case timed twice
+
+
+def test_case_targets_are_the_stated_bars():
+    assert bench.case_target("q8", 1) == ("hbm_frac", 0.70)
+    assert bench.case_target("q8", 16) == ("hbm_frac", 0.70)
+    assert bench.case_target("q4", 8) == ("hbm_frac", 0.70)
+    assert bench.case_target("w8a8", 4096) == ("tensor_frac", 0.60)
+    assert bench.case_target("q8", 432) is None and bench.case_target("w8a8", 432) is None
+
+
+def test_roof_entry_picks_the_binding_roof():
+    R = bench.roofs({"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0})
+    assert R == {"f16": 1600.0, "i8": 3200.0, "hbm": 6000.0}
+    # weight-bound: 4 MB and 8 MFLOP in 1 us -> 4 TB/s, HBM-bound
+    d = bench.roof_entry(8e6, 4e6, 1e-6, R["f16"], R["hbm"])
+    assert d["bound"] == "hbm" and d["frac"] == pytest.approx(4000 / 6000)
+    # compute-bound: 8 GFLOP, 10 MB in 10 us -> 800 TFLOP/s
+    d = bench.roof_entry(8e9, 10e6, 10e-6, R["f16"], R["hbm"])
+    assert d["bound"] == "tensor" and d["frac"] == pytest.approx(800 / 1600)
+    d = bench.roof_entry(0.0, 3e6, 1e-6, R["f16"], R["hbm"])   # a quantiser: bytes only
+    assert d["bound"] == "hbm" and "tops" not in d
+
+
+def test_fp16_rung_account():
+    acc = bench.step_account()
+    params = 1536 * 4608 + 1536 * 1536 + 1536 * 6144 + 6144 * 1536
+    assert acc["f16"][0] == acc["q8"][0]
+    xy = sum(2 * 432 * k + 2 * 432 * n for _, k, n in bench.LINEARS)
+    assert acc["f16"][1] == 8 * (24 * (2 * params + xy) + 4 * 1536)

@@ -102,10 +102,20 @@ def test_act_quant_bit_exact(M, K):
 # ------------------------------------------------------------ int8 GEMM ---
 
 def _w8a8_inputs(M, N, K, key):
+    """GPU pack and activation codes, each first checked bit for bit against
+    the oracle's own (so the GEMM parity below runs pack -> GEMM end to end
+    against the oracle's pack -> GEMM)."""
     W = synthetic.weight(f"{key}/W", N, K)
     X = synthetic.activation(key, M, K, outlier_channel_frac=0.01)
     Wq, sw = aq.qpack("q8", W.cuda())
     Xq, sx = aq.act_quant(X.cuda())
+    rq, rs = oracle.pack_q8(W.numpy())
+    assert np.array_equal(Wq.cpu().numpy(), rq) and np.array_equal(sw.cpu().numpy().view(np.uint32),
+                                                                   rs.view(np.uint32))
+    if M * K <= 4096 * 6144:
+        xq, xs = oracle.act_quant(X.numpy())
+        assert np.array_equal(Xq.cpu().numpy(), xq) and np.array_equal(sx.cpu().numpy().view(np.uint32),
+                                                                       xs.view(np.uint32))
     return X, W, Xq, sx, Wq, sw
 
 
@@ -178,6 +188,38 @@ def test_w8a8_exact_fp16_ties_round_to_even(M, N, K, bias, steer):
     assert np.array_equal(got, ref), (got != ref).sum()
 
 
+@pytest.mark.parametrize("M,N", [(1, 16), (4096, 1280)])   # split-K and persistent epilogues
+@pytest.mark.parametrize("term", ["bias", "steer"])
+def test_w8a8_just_below_the_overflow_midpoint(M, N, term):
+    """acc * s_x * s_w = 65520 exactly (the midpoint between 65504 and
+    overflow) plus a negative bias of 2^-14 (or the same through alpha*v): in
+    fp32 the sum rounds to 65520 itself, and converting that to fp16 ties up
+    to infinity, but the exact value lies below the midpoint and rounds to
+    65504. Rows alternate with the exact midpoint (bias / steer 0 there:
+    infinity is right) to keep both sides covered."""
+    K = 512
+    xc = np.zeros((M, K)); wc = np.zeros((N, K))
+    xc[:, :5] = 127; xc[:, 5] = -12                # s_x = 1
+    wc[:, :4] = 127; wc[:, 4] = 8; wc[:, 5] = 1    # s_w = 1; acc = 4*127^2 + 127*8 - 12 = 65520
+    X = torch.from_numpy(xc.astype(np.float16))
+    W = torch.from_numpy(wc.astype(np.float16))
+    Wq, sw = aq.qpack("q8", W.cuda())
+    Xq, sx = aq.act_quant(X.cuda())
+    assert (sx == 1).all() and (sw == 1).all()
+    assert (aq.qgemm_s32(Xq, Wq) == 65520).all()
+    small = np.where(np.arange(N) % 2 == 0, -2.0 ** -14, 0.0)
+    if term == "bias":
+        b, v, alpha = small.astype(np.float16), None, 0.0
+    else:
+        b, v, alpha = None, (small * 2.0).astype(np.float32), 0.5      # alpha*v = small, exactly
+    Y = aq.qgemm("w8a8", Xq, Wq, sw, sx=sx, bias=None if b is None else torch.from_numpy(b).cuda(),
+                 steer_vec=None if v is None else torch.from_numpy(v).cuda(), alpha=alpha)
+    rows = sample_rows(M, 32)
+    ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(), b, v, alpha, rows=rows)
+    assert (ref[:, 0] == 0x7BFF).all() and (ref[:, 1] == 0x7C00).all()
+    assert np.array_equal(Y.cpu().numpy().view(np.uint16)[rows], ref)
+
+
 def test_w8a8_large_accumulators_take_exact_path():
     """|acc| >= 2^22 (all codes +-127 over K = 4096) and exact fp16 results
     exercise the kernel's fp64 branch; sign patterns vary per row/column."""
@@ -197,7 +239,8 @@ def test_w8a8_large_accumulators_take_exact_path():
     assert np.array_equal(Y.cpu().numpy().view(np.uint16), ref)
 
 
-@pytest.mark.parametrize("M,N,K", [(4096, 6144, 1536), (4096, 1536, 6144), (4096, 4608, 1536)])
+@pytest.mark.parametrize("M,N,K", [(4096, 6144, 1536), (4096, 1536, 6144), (4096, 4608, 1536),
+                                   (4096, 1536, 1536)])
 def test_w8a8_full_size_sampled(M, N, K):
     key = f"gpu/w8a8f/{M}x{N}x{K}"
     X, W, Xq, sx, Wq, sw = _w8a8_inputs(M, N, K, key)
@@ -221,10 +264,15 @@ def _wo(fmt, M, N, K, key, bias=False, steer=False, rows=None, outliers=0.0):
     Wq, sc = aq.qpack(fmt, W.cuda())
     Y = aq.qgemm(fmt, X.cuda(), Wq, sc, bias=None if b is None else b.cuda(),
                  steer_vec=None if v is None else v.cuda(), alpha=alpha)
+    # the oracle's own pack: the GPU's must equal it, and the reference is
+    # computed from it (pack -> GEMM end to end on both sides)
+    rq, rs = oracle.pack_q8(W.numpy()) if fmt == "q8" else oracle.pack_q4(W.numpy())
     scn = sc.cpu().numpy()
-    ref = oracle.wo_ref(fmt, X.numpy(), Wq.cpu().numpy(), scn if fmt == "q8" else scn.view(np.uint16),
-                        None if b is None else b.numpy(), None if v is None else v.numpy(), alpha,
-                        rows=rows)
+    assert np.array_equal(Wq.cpu().numpy(), rq)
+    assert np.array_equal(scn.view(np.uint32) if fmt == "q8" else scn.view(np.uint16),
+                          rs.view(np.uint32) if fmt == "q8" else rs)
+    ref = oracle.wo_ref(fmt, X.numpy(), rq, rs, None if b is None else b.numpy(),
+                        None if v is None else v.numpy(), alpha, rows=rows)
     y = f16np(Y)
     return (y if rows is None else y[rows]), ref
 
@@ -255,7 +303,9 @@ def test_q8_d1024_block(name, M):
     Wq, s = aq.qpack("q8", W.cuda())
     Y = aq.qgemm("q8", X.cuda(), Wq, s)
     rows = sample_rows(M, 24)
-    ref = oracle.wo_ref("q8", X.numpy(), Wq.cpu().numpy(), s.cpu().numpy(), rows=rows)
+    rq, rs = oracle.pack_q8(W.numpy())
+    assert np.array_equal(Wq.cpu().numpy(), rq) and np.array_equal(s.cpu().numpy(), rs)
+    ref = oracle.wo_ref("q8", X.numpy(), rq, rs, rows=rows)
     check_wo(f16np(Y)[rows], ref)
 
 
@@ -274,7 +324,9 @@ def test_q4_d1536_block(name, M):
     P, S = aq.qpack("q4", W.cuda())
     Y = aq.qgemm("q4", X.cuda(), P, S)
     rows = sample_rows(M, 16)
-    ref = oracle.wo_ref("q4", X.numpy(), P.cpu().numpy(), S.cpu().numpy().view(np.uint16), rows=rows)
+    rp, rs = oracle.pack_q4(W.numpy())
+    assert np.array_equal(P.cpu().numpy(), rp) and np.array_equal(S.cpu().numpy().view(np.uint16), rs)
+    ref = oracle.wo_ref("q4", X.numpy(), rp, rs, rows=rows)
     check_wo(f16np(Y)[rows], ref)
 
 
@@ -443,11 +495,12 @@ def test_dependent_chain_in_replay_launch_configuration(graph):
 def test_bench_replay_outputs_match_oracle():
     """bench.py's own workload and launches: bench.Replay's CUDA graphs (24
     blocks x 4 linears x 8 steps per precision at M = 432, steering on block
-    12's out-projection), replayed precision by precision; then sampled
-    outputs of blocks 0, 12 and 23 against the oracle: q8 and q4 within the
-    weight-only tolerance, W8A8 bit-exact."""
+    12's out-projection with the strength read from the device schedule),
+    replayed precision by precision, from both input buffers; then sampled
+    outputs of blocks 0, 12 and 23 against the oracle: q8, q4 and fp16 within
+    the weight-only tolerance, W8A8 bit-exact."""
     import bench
-    rep = bench.Replay(torch.device("cuda", torch.cuda.current_device()))
+    rep = bench.Replay(torch.device("cuda", torch.cuda.current_device()), buffers=2, fp16=True)
     rep.capture()
     rows = sample_rows(bench.M, 4)
     blocks = (0, synthetic.REPLAY_STEER_BLOCK, bench.BLOCKS - 1)
@@ -457,34 +510,46 @@ def test_bench_replay_outputs_match_oracle():
         on = b == synthetic.REPLAY_STEER_BLOCK and name == "out"
         return (v, synthetic.REPLAY_ALPHA) if on else (None, 0.0)
 
-    def replay(*kinds):
+    def replay(buf, *kinds):
+        for kind in kinds:
+            for key in rep.y.get(kind.replace("_gemm", ""), {}):
+                rep.y[kind.replace("_gemm", "")][key].fill_(float("nan"))   # no stale result passes
         with torch.cuda.stream(rep.stream):
             for kind in kinds:
-                rep.graphs[kind].replay()
+                rep.graphs[kind, buf if kind != "w8a8_gemm" else 0].replay()
         torch.cuda.synchronize()
 
-    replay("q8")
-    for b in blocks:
-        for name, k, n in bench.LINEARS:
-            x = rep.x_host[b, name].numpy()
-            Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
-            vv, a = steer(b, name)
-            check_wo(f16np(rep.y[b, name])[rows], oracle.wo_ref("q8", x, Wq, sw, None, vv, a, rows=rows))
-    replay("act_quant", "w8a8_gemm")
-    for b in blocks:
-        for name, k, n in bench.LINEARS:
-            x = rep.x_host[b, name].numpy()
-            Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
-            vv, a = steer(b, name)
-            ref = oracle.w8a8(x, Wq, sw, None, vv, a, rows=rows)
-            assert np.array_equal(f16np(rep.y[b, name]).view(np.uint16)[rows], ref), (b, name)
-    replay("q4")
-    for b in blocks:
-        for name, k, n in bench.LINEARS:
-            x = rep.x_host[b, name].numpy()
-            P, S = rep.q4[b, name]
-            vv, a = steer(b, name)
-            ref = oracle.wo_ref("q4", x, P.cpu().numpy(), S.cpu().numpy().view(np.uint16), None, vv, a,
-                                rows=rows)
-            check_wo(f16np(rep.y[b, name])[rows], ref)
+    for buf in (0, 1):
+        replay(buf, "q8")
+        for b in blocks:
+            for name, k, n in bench.LINEARS:
+                x = rep.x_host[b, name].numpy()
+                Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
+                vv, a = steer(b, name)
+                check_wo(f16np(rep.y["q8"][b, name])[rows],
+                         oracle.wo_ref("q8", x, Wq, sw, None, vv, a, rows=rows))
+        replay(buf, "act_quant", "w8a8_gemm")
+        for b in blocks:
+            for name, k, n in bench.LINEARS:
+                x = rep.x_host[b, name].numpy()
+                Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
+                vv, a = steer(b, name)
+                ref = oracle.w8a8(x, Wq, sw, None, vv, a, rows=rows)
+                assert np.array_equal(f16np(rep.y["w8a8"][b, name]).view(np.uint16)[rows], ref), (b, name)
+        replay(buf, "q4")
+        for b in blocks:
+            for name, k, n in bench.LINEARS:
+                x = rep.x_host[b, name].numpy()
+                P, S = rep.q4[b, name]
+                vv, a = steer(b, name)
+                ref = oracle.wo_ref("q4", x, P.cpu().numpy(), S.cpu().numpy().view(np.uint16), None, vv, a,
+                                    rows=rows)
+                check_wo(f16np(rep.y["q4"][b, name])[rows], ref)
+        replay(buf, "f16")
+        for b in blocks:
+            for name, k, n in bench.LINEARS:
+                x = rep.x_host[b, name].numpy()
+                vv, a = steer(b, name)
+                ref = oracle.f16_ref(x, rep.w16[b, name].cpu().numpy(), None, vv, a, rows=rows)
+                check_wo(f16np(rep.y["f16"][b, name])[rows], ref)
     rep.aq.device_status(rep.stream)
