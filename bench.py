@@ -700,6 +700,10 @@ def _case_inputs(case, name, n, k, m):
     if name == "tiny":
         d = synthetic.tiny_q8()
         return d["W"], d["X"]
+    if not name:   # an arbitrary shape (--case): the same distributions, keyed by the shape
+        return (synthetic.weight(f"case/{n}x{k}", n, k, outlier_frac=0.001 if case.endswith("q4") else 0.0),
+                synthetic.activation(f"case/{max(m, 1)}x{k}", max(m, 1), k,
+                                     outlier_channel_frac=0.01 if case == "w8a8" else 0.0))
     if case == "q8":
         return synthetic.q8_block_d1024(name, m)
     if case in ("w8a8", "pack_q8"):

@@ -16,6 +16,7 @@
 #include "ptx.cuh"
 #include "qgemm.cuh"
 #include "quant_kernels.cuh"
+#include "smallm.cuh"
 
 #define ARIA_API extern "C" __attribute__((visibility("default")))
 
@@ -325,6 +326,174 @@ aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap
   return ARIA_OK;
 }
 
+// ------------------------------------------------------------- few tokens ---
+// Plan of the few-token weight-only GEMM (smallm_kernel): the smallest
+// cluster size S (K split) that keeps each warp's activation chunks in
+// registers and the activations read per CTA at or below 32 KB, with the
+// rows divided over as many clusters as the SMs hold. False when no plan
+// fits (then the tensor-core kernel runs).
+struct SmallPlan {
+  aria::SmallParams p;
+  int grid = 0, tb = 1, ch = 8;
+  size_t smem = 0;
+};
+
+constexpr int64_t kSmallMaxTokens = 16;
+constexpr size_t kSmallSmemBudget = 110 * 1024;  // two CTAs per SM
+
+template <int KIND, int TB, int CH, int GP>
+int small_max_clusters(int size, size_t smem) {
+  static std::mutex mu;
+  static int cache_dev[64], cache_size[64], cache_n[64];
+  static size_t cache_smem[64];
+  static int used = 0;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> g(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache_dev[i] == dev && cache_size[i] == size && cache_smem[i] == smem) return cache_n[i];
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(size, 1, 1);
+  cfg.blockDim = dim3(aria::kSmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = size;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, aria::smallm_kernel<KIND, TB, CH, GP>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (used < 64) {
+    cache_dev[used] = dev;
+    cache_size[used] = size;
+    cache_smem[used] = smem;
+    cache_n[used] = n;
+    ++used;
+  }
+  return n;
+}
+
+// shared-memory layout of a plan with `clusters` clusters of S CTAs
+bool small_layout(int kind, int64_t M, int64_t N, int64_t K, int S, int clusters, int tb, int gp,
+                  aria::SmallParams* p, size_t* smem) {
+  using namespace aria;
+  const int num = kind == kF16 ? 2 : 1, den = kind == kQ4 ? 2 : 1;
+  p->S = S;
+  p->kslice = static_cast<int>(K / S);
+  p->rows_base = static_cast<int>(N / clusters);
+  p->rows_rem = static_cast<int>(N % clusters);
+  const int rmax = p->rows_base + (p->rows_rem ? 1 : 0);
+  p->r_pad = (rmax + 15) / 16 * 16;
+  const uint32_t slice = static_cast<uint32_t>(p->kslice) * num / den;
+  p->wrow = slice + 16;
+  auto up = [](uint64_t v, uint64_t a) { return (v + a - 1) / a * a; };
+  uint64_t off = up(static_cast<uint64_t>(rmax) * p->wrow, 128);
+  p->off_sc = static_cast<uint32_t>(off);
+  if (kind == kQ4) off = up(off + static_cast<uint64_t>(rmax) * (p->kslice / 16), 128);
+  p->off_red = static_cast<uint32_t>(off);
+  off += static_cast<uint64_t>(kSmWarps) * tb * 8 * sm_red_stride(gp) * 4;
+  p->off_part = static_cast<uint32_t>(up(off, 128));
+  off = p->off_part + (S > 1 ? static_cast<uint64_t>(tb) * 8 * (p->r_pad + 4) * 4 : 0);
+  p->off_bar = static_cast<uint32_t>(up(off, 16));
+  *smem = p->off_bar + 16;
+  (void)M;
+  return *smem <= kSmallSmemBudget;
+}
+
+template <int KIND, int TB, int CH, int GP>
+bool plan_small_t(int64_t M, int64_t N, int64_t K, SmallPlan* out) {
+  using namespace aria;
+  const DevInfo di = dev_info();
+  const int unit = KIND == kQ4 ? 256 : 64;
+  if (K % unit) return false;
+  int best_s = 0;
+  for (int S = 1; S <= 8; ++S) {
+    if (K % (static_cast<int64_t>(S) * unit)) continue;
+    const int64_t kslice = K / S;
+    if ((kslice / 64 + kSmWarps - 1) / kSmWarps > CH) continue;  // activation chunks in registers
+    best_s = S;
+    if (M * kslice * 2 <= 32768) break;  // activations read per CTA: small enough
+  }
+  if (best_s == 0) return false;
+  const int S = best_s;
+  int clusters = static_cast<int>(std::min<int64_t>(di.sms / S, N));
+  SmallParams p{};
+  size_t smem = 0;
+  if (!small_layout(KIND, M, N, K, S, clusters, TB, GP, &p, &smem)) return false;
+  if (S > 1) {
+    const int fit = small_max_clusters<KIND, TB, CH, GP>(S, smem);
+    if (fit < 1) return false;
+    if (fit < clusters) {
+      clusters = fit;
+      if (!small_layout(KIND, M, N, K, S, clusters, TB, GP, &p, &smem)) return false;
+    }
+  }
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  out->p = p;
+  out->grid = clusters * S;
+  out->tb = TB;
+  out->ch = CH;
+  out->smem = smem;
+  return true;
+}
+
+bool plan_small(int kind, int64_t M, int64_t N, int64_t K, SmallPlan* out) {
+  using namespace aria;
+  if (M > kSmallMaxTokens) return false;
+  const bool two = M > 8;
+  switch (kind) {
+    case kQ8: return two ? plan_small_t<kQ8, 2, 4, 2>(M, N, K, out) : plan_small_t<kQ8, 1, 6, 4>(M, N, K, out);
+    case kQ4: return two ? plan_small_t<kQ4, 2, 4, 2>(M, N, K, out) : plan_small_t<kQ4, 1, 6, 4>(M, N, K, out);
+    case kF16: return two ? plan_small_t<kF16, 2, 4, 2>(M, N, K, out) : plan_small_t<kF16, 1, 6, 4>(M, N, K, out);
+  }
+  return false;
+}
+
+template <int KIND, int TB, int CH, int GP>
+aria_status launch_small_t(const SmallPlan& pl, cudaStream_t st) {
+  auto kfn = aria::smallm_kernel<KIND, TB, CH, GP>;
+  static bool attr_done[kMaxDevices] = {};
+  static std::mutex attr_mu;
+  aria_status as = opt_in_smem(kfn, attr_done, attr_mu);
+  if (as != ARIA_OK) return as;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
+  cfg.blockDim = dim3(aria::kSmThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  cfg.numAttrs = 0;
+  if (pl.p.S > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.p.S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+    cfg.attrs = attr;
+  }
+  set_pdl(cfg, attr);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, pl.p);
+  if (e != cudaSuccess) return cuda_fail(e, "few-token GEMM launch");
+  return ARIA_OK;
+}
+
+aria_status launch_small(int kind, const SmallPlan& pl, cudaStream_t st) {
+  using namespace aria;
+  const bool two = pl.tb == 2;
+  switch (kind) {
+    case kQ8: return two ? launch_small_t<kQ8, 2, 4, 2>(pl, st) : launch_small_t<kQ8, 1, 6, 4>(pl, st);
+    case kQ4: return two ? launch_small_t<kQ4, 2, 4, 2>(pl, st) : launch_small_t<kQ4, 1, 6, 4>(pl, st);
+    case kF16: return two ? launch_small_t<kF16, 2, 4, 2>(pl, st) : launch_small_t<kF16, 1, 6, 4>(pl, st);
+  }
+  return fail(ARIA_ERR_INVALID_ARG, "unknown kind");
+}
+
 aria_status check_gemm_shape(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
     return fail(ARIA_ERR_INVALID_ARG, "sizes must be positive and < 2^31 (M=%lld N=%lld K=%lld)",
@@ -440,6 +609,20 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
   if ((kind == kW8A8 || kind == kS32) && K * 127 * 127 > INT32_MAX)
     return fail(ARIA_ERR_UNSUPPORTED, "int8 GEMM needs K * 127^2 < 2^31 (K <= %lld), got K=%lld",
                 (long long)(INT32_MAX / (127 * 127)), (long long)K);
+  // a handful of tokens: the weight-streaming kernel, when its plan fits
+  SmallPlan sp;
+  if (plan_small(kind, M, N, K, &sp)) {
+    sp.p.W = static_cast<const uint8_t*>(Wq);
+    sp.p.Wsc = kind == kQ4 ? static_cast<const __half*>(scales) : nullptr;
+    sp.p.sw = kind == kQ8 ? static_cast<const float*>(scales) : nullptr;
+    sp.p.X = static_cast<const __half*>(X);
+    sp.p.bias = static_cast<const __half*>(bias);
+    sp.p.steer = (steer && (alpha_dev || alpha != 0.0f)) ? steer : nullptr;
+    sp.p.alpha = sp.p.steer ? alpha : 0.0f;
+    sp.p.alpha_dev = sp.p.steer ? alpha_dev : nullptr;
+    sp.p.Y = static_cast<__half*>(Y);
+    return launch_small(kind, sp, st);
+  }
   Plan pl;
   if ((s = plan_gemm(kind, M, N, K, &pl)) != ARIA_OK) return s;
   CUtensorMap tw, ts, tx;
