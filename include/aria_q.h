@@ -38,7 +38,9 @@
  *   - Non-finite inputs are outside the contract (not checked).
  *   - The library allocates no device memory, makes no host-device copies
  *     inside the entry points below, and is safe to call while a stream is
- *     being captured into a CUDA graph (aria_device_status excepted).
+ *     being captured into a CUDA graph (aria_device_status excepted). The
+ *     one entry point that needs scratch memory (aria_qgemm_w8a8_fused)
+ *     takes it from the caller.
  */
 #ifndef ARIA_Q_H
 #define ARIA_Q_H
@@ -172,6 +174,47 @@ aria_status aria_qgemm_steer_dev(aria_format fmt, int group, int64_t M, int64_t 
                                  const void *X, const float *sx, const void *Wq,
                                  const void *scales, const void *bias, const float *steer_vec,
                                  const float *alpha_dev, void *Y, void *stream);
+
+/*
+ * aria_w8a8_workspace_size -- bytes of the workspace aria_qgemm_w8a8_fused
+ * needs for M tokens of K features: 256 + 4*M rounded up to 256 + M*K.
+ * Errors: INVALID_ARG (NULL output, M or K outside [1, 2^31)).
+ */
+aria_status aria_w8a8_workspace_size(int64_t M, int64_t K, size_t *bytes);
+
+/*
+ * aria_qgemm_w8a8_fused -- the W8A8 linear from fp16 activations in one
+ * launch: the per-token int8 quantisation of X (exactly aria_act_quant's
+ * rule and bits) runs inside the GEMM kernel, then the integer-tensor-core
+ * GEMM and the epilogue of aria_qgemm(ARIA_FMT_W8A8) ("Results": W8A8 is
+ * 8-bit arithmetic on integer tensor cores; the activations are quantised
+ * per token).
+ *   X          device fp16 [M,K] row-major (not quantised).
+ *   Wq, sw     device, the Q8 pack (int8 [N,K], fp32 [N]).
+ *   bias, steer_vec, alpha  as for aria_qgemm; alpha_dev, if not NULL, a
+ *              device fp32 scalar (4-byte aligned) used instead of alpha, as
+ *              in aria_qgemm_steer_dev.
+ *   Y          device output fp16 [M,N]: the same bytes as aria_act_quant
+ *              followed by aria_qgemm(ARIA_FMT_W8A8).
+ *   workspace  caller-owned device memory, 256-byte aligned, at least
+ *              aria_w8a8_workspace_size(M, K) bytes (INVALID_ARG otherwise).
+ *              Its first 256 bytes hold a grid barrier and must be zero
+ *              before the first call; every successful call leaves them
+ *              zero. After the call the workspace holds the token scales
+ *              (fp32 [M] at byte 256) and the codes (int8 [M,K] at byte
+ *              256 + 4*M rounded up to 256), as aria_act_quant would write
+ *              them. Calls that share a workspace must not overlap on the
+ *              GPU (one stream, or ordered by events).
+ *   The kernel's CTAs meet at a grid-wide barrier after quantising their
+ *   share of the rows; its wait is bounded: if it runs out, the device
+ *   status word reports ARIA_ERR_TIMEOUT and the workspace's first 256 bytes
+ *   must be zeroed again before the next call.
+ * Shape rules and stream order as for aria_qgemm(ARIA_FMT_W8A8).
+ */
+aria_status aria_qgemm_w8a8_fused(int64_t M, int64_t N, int64_t K, const void *X, const void *Wq,
+                                  const float *sw, const void *bias, const float *steer_vec,
+                                  float alpha, const float *alpha_dev, void *Y, void *workspace,
+                                  size_t workspace_bytes, void *stream);
 
 /*
  * aria_qgemm_s32 -- the W8A8 integer GEMM alone: C[m,n] = sum_k Xq[m,k]*Wq[n,k]

@@ -30,8 +30,8 @@ STATUS = {0: "ARIA_OK", 1: "ARIA_ERR_INVALID_ARG", 2: "ARIA_ERR_UNSUPPORTED",
           3: "ARIA_ERR_MISALIGNED", 4: "ARIA_ERR_CUDA", 5: "ARIA_ERR_TIMEOUT"}
 FORMATS = {"q8": 1, "q4": 2, "w8a8": 3, "f16": 4}
 API = ("aria_status_string", "aria_last_error_message", "aria_qpack_size", "aria_qpack",
-       "aria_act_quant", "aria_qgemm", "aria_qgemm_steer_dev", "aria_qgemm_s32",
-       "aria_device_status")
+       "aria_act_quant", "aria_qgemm", "aria_qgemm_steer_dev", "aria_w8a8_workspace_size",
+       "aria_qgemm_w8a8_fused", "aria_qgemm_s32", "aria_device_status")
 
 
 class AriaError(RuntimeError):
@@ -60,6 +60,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "aria_act_quant": ([P, I64, I64, P, P, P], I),
         "aria_qgemm": ([I, I, I64, I64, I64, P, P, P, P, P, P, ctypes.c_float, P, P], I),
         "aria_qgemm_steer_dev": ([I, I, I64, I64, I64, P, P, P, P, P, P, P, P, P], I),
+        "aria_w8a8_workspace_size": ([I64, I64, P], I),
+        "aria_qgemm_w8a8_fused": ([I64, I64, I64, P, P, P, P, P, ctypes.c_float, P, P, P,
+                                   ctypes.c_size_t, P], I),
         "aria_qgemm_s32": ([I64, I64, I64, P, P, P, P], I),
         "aria_device_status": ([P], I),
     }
@@ -252,6 +255,62 @@ def qgemm(fmt: str, X: torch.Tensor, Wq: torch.Tensor, scales, sx=None,
                                             _stream(stream)))
         else:
             _check(lib.aria_qgemm(*args, float(alpha), _dev(Y, "out"), _stream(stream)))
+    return Y
+
+
+def w8a8_workspace_size(M: int, K: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().aria_w8a8_workspace_size(M, K, ctypes.byref(n)))
+    return n.value
+
+
+def w8a8_workspace(M: int, K: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace for qgemm_w8a8_fused (uint8, 256-byte aligned:
+    the caching allocator's blocks are)."""
+    ws = torch.zeros(w8a8_workspace_size(M, K), dtype=torch.uint8, device=device)
+    if ws.data_ptr() % 256:
+        raise RuntimeError("workspace is not 256-byte aligned")
+    return ws
+
+
+def workspace_codes(ws: torch.Tensor, M: int, K: int):
+    """Views of the token scales fp32 [M] and codes int8 [M,K] that a fused
+    call leaves in its workspace (the layout of include/aria_q.h)."""
+    sx_bytes = (4 * M + 255) // 256 * 256
+    sx = ws[256:256 + 4 * M].view(torch.float32)
+    xq = ws[256 + sx_bytes:256 + sx_bytes + M * K].view(torch.int8).view(M, K)
+    return xq, sx
+
+
+def qgemm_w8a8_fused(X: torch.Tensor, Wq: torch.Tensor, sw: torch.Tensor, bias=None, steer_vec=None,
+                     alpha: float = 0.0, alpha_dev=None, out=None, workspace=None, stream=None):
+    """W8A8 from fp16 X [M,K] in one launch: per-token quantisation inside the
+    GEMM kernel (include/aria_q.h, aria_qgemm_w8a8_fused). ``workspace``: a
+    zero-filled uint8 tensor of w8a8_workspace_size(M, K) bytes (see
+    w8a8_workspace); calls sharing one must not overlap on the GPU."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _expect(X, "X", (M, K), torch.float16)
+    _expect(Wq, "Wq", (N, K), torch.int8)
+    _expect(sw, "scales", (N,), torch.float32)
+    _expect(bias, "bias", (N,), torch.float16)
+    _expect(steer_vec, "steer_vec", (N,), torch.float32)
+    if alpha_dev is not None and (alpha_dev.numel() != 1 or alpha_dev.dtype != torch.float32):
+        raise TypeError("alpha_dev must be one float32 element")
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=X.device)
+    _expect(Y, "out", (M, N), torch.float16)
+    if workspace is None:
+        raise ValueError("qgemm_w8a8_fused needs a workspace (w8a8_workspace(M, K, device))")
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous uint8 tensor")
+    same_device(X=X, Wq=Wq, scales=sw, bias=bias, steer_vec=steer_vec, out=Y, workspace=workspace,
+                alpha_dev=alpha_dev)
+    with _on(X.device):
+        _check(load_library().aria_qgemm_w8a8_fused(
+            M, N, K, _dev(X, "X", torch.float16), _dev(Wq, "Wq", torch.int8), _dev(sw, "scales"),
+            _dev(bias, "bias", torch.float16), _dev(steer_vec, "steer_vec", torch.float32),
+            float(alpha), None if alpha_dev is None else _dev(alpha_dev, "alpha_dev"),
+            _dev(Y, "out"), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)))
     return Y
 
 

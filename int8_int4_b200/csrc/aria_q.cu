@@ -597,10 +597,34 @@ ARIA_API aria_status aria_act_quant(const void* X, int64_t M, int64_t K, int8_t*
   return ARIA_OK;
 }
 
+// Workspace of the fused W8A8 call: [0, 256) the grid barrier {arrivals,
+// generation}; then the token scales fp32 [M]; then the codes int8 [M,K], at
+// 256-byte aligned offsets (TMA reads the codes).
+struct FusedWs {
+  unsigned* gbar;
+  float* sx;
+  int8_t* xq;
+};
+
+constexpr size_t kWsHeader = 256;
+
+size_t fused_ws_bytes(int64_t M, int64_t K) {
+  const size_t sx = (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
+  return kWsHeader + sx + static_cast<size_t>(M) * static_cast<size_t>(K);
+}
+
+FusedWs fused_ws(void* ws, int64_t M) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t sx = (static_cast<size_t>(M) * 4 + 255) / 256 * 256;
+  return FusedWs{reinterpret_cast<unsigned*>(b), reinterpret_cast<float*>(b + kWsHeader),
+                 reinterpret_cast<int8_t*>(b + kWsHeader + sx)};
+}
+
 static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const void* X,
                               const float* sx, const void* Wq, const void* scales,
                               const void* bias, const float* steer, float alpha,
-                              const float* alpha_dev, void* Y, cudaStream_t st) {
+                              const float* alpha_dev, void* Y, cudaStream_t st,
+                              const void* xf16 = nullptr, const FusedWs* ws = nullptr) {
   using namespace aria;
   aria_status s = check_gemm_shape(M, N, K);
   if (s != ARIA_OK) return s;
@@ -611,7 +635,7 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
                 (long long)(INT32_MAX / (127 * 127)), (long long)K);
   // a handful of tokens: the weight-streaming kernel, when its plan fits
   SmallPlan sp;
-  if (plan_small(kind, M, N, K, &sp)) {
+  if (!xf16 && plan_small(kind, M, N, K, &sp)) {
     sp.p.W = static_cast<const uint8_t*>(Wq);
     sp.p.Wsc = kind == kQ4 ? static_cast<const __half*>(scales) : nullptr;
     sp.p.sw = kind == kQ8 ? static_cast<const float*>(scales) : nullptr;
@@ -656,6 +680,13 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
   pl.p.alpha = pl.p.steer ? alpha : 0.0f;
   pl.p.alpha_dev = pl.p.steer ? alpha_dev : nullptr;
   pl.p.Y = Y;
+  if (xf16) {  // W8A8 with the activation quantisation in this launch
+    pl.p.xf16 = static_cast<const __half*>(xf16);
+    pl.p.xq_ws = ws->xq;
+    pl.p.sx_ws = ws->sx;
+    pl.p.gbar = ws->gbar;
+    pl.p.sx = ws->sx;
+  }
   switch (kind) {
     case kQ8: return launch_gemm<kQ8>(pl, tw, tw, tx, st);
     case kQ4: return launch_gemm<kQ4>(pl, tw, ts, tx, st);
@@ -721,6 +752,37 @@ ARIA_API aria_status aria_qgemm_steer_dev(aria_format fmt, int group, int64_t M,
     return fail(ARIA_ERR_MISALIGNED, "alpha_dev must be 4-byte aligned");
   return qgemm_impl(kind, M, N, K, X, sx, Wq, scales, bias, steer_vec, 0.0f, alpha_dev, Y,
                     static_cast<cudaStream_t>(stream));
+}
+
+ARIA_API aria_status aria_w8a8_workspace_size(int64_t M, int64_t K, size_t* bytes) {
+  if (!bytes) return fail(ARIA_ERR_INVALID_ARG, "NULL output pointer");
+  if (M < 1 || K < 1 || M > kMaxDim || K > kMaxDim)
+    return fail(ARIA_ERR_INVALID_ARG, "M and K must be in [1, 2^31)");
+  *bytes = fused_ws_bytes(M, K);
+  return ARIA_OK;
+}
+
+ARIA_API aria_status aria_qgemm_w8a8_fused(int64_t M, int64_t N, int64_t K, const void* X,
+                                           const void* Wq, const float* sw, const void* bias,
+                                           const float* steer_vec, float alpha,
+                                           const float* alpha_dev, void* Y, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!X || !Wq || !sw || !Y || !workspace) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  for (const void* q : {X, static_cast<const void*>(Wq), static_cast<const void*>(sw), bias,
+                        static_cast<const void*>(steer_vec), static_cast<const void*>(Y)})
+    if (q && !aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(ARIA_ERR_MISALIGNED, "the workspace must be 256-byte aligned");
+  if (alpha_dev && (reinterpret_cast<uintptr_t>(alpha_dev) & 3u))
+    return fail(ARIA_ERR_MISALIGNED, "alpha_dev must be 4-byte aligned");
+  aria_status s = check_gemm_shape(M, N, K);
+  if (s != ARIA_OK) return s;
+  if (workspace_bytes < fused_ws_bytes(M, K))
+    return fail(ARIA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                fused_ws_bytes(M, K));
+  const FusedWs ws = fused_ws(workspace, M);
+  return qgemm_impl(aria::kW8A8, M, N, K, ws.xq, ws.sx, Wq, sw, bias, steer_vec, alpha, alpha_dev, Y,
+                    static_cast<cudaStream_t>(stream), X, &ws);
 }
 
 ARIA_API aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t* Xq,

@@ -40,6 +40,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quant_kernels.cuh"
 
 namespace aria {
 
@@ -67,6 +68,14 @@ struct GemmParams {
   const float* steer;     // [N] or null (null also when a host alpha is 0)
   float alpha;
   const float* alpha_dev; // device alpha, read after the dependency wait; null: use `alpha`
+  // W8A8 with the activation quantisation in the same launch (null: X is
+  // already quantised): fp16 X, and the workspace that receives its codes
+  // and token scales (read back through tmX and sx) and holds the grid
+  // barrier {arrivals, generation}
+  const __half* xf16;
+  int8_t* xq_ws;
+  float* sx_ws;
+  unsigned* gbar;
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
@@ -436,6 +445,82 @@ __device__ __forceinline__ void epilogue_chunk_store(int c, int nb, int m0, int 
     }
 }
 
+// ----------------------------------------------- fused activation quant ---
+// "Results" (aria project page): W8A8 quantises the activations per token to
+// 8 bits. In the fused form every CTA of the GEMM quantises a share of the
+// token rows (one warp per row: absmax, s = absmax / 127 as an IEEE fp32
+// quotient, codes rounded half-to-even -- the same steps and bits as
+// row_quant_i8_kernel) into the workspace, publishes the stores to the
+// async proxy, and meets the other CTAs at a grid-wide barrier; the MMA
+// pipeline then loads the codes with TMA. The grid never exceeds the SMs
+// and each CTA fills one SM, so all CTAs are resident together once the
+// preceding kernel has finished. The barrier is a sense-reversal barrier:
+// the last CTA to arrive resets the count to zero and advances the
+// generation, so the workspace is ready for the next call. Waiting is
+// bounded (kWaitLimitNs); on timeout the status word records it.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __noinline__ bool grid_barrier(unsigned* gbar, unsigned ctas, volatile int* abort) {
+  unsigned* count = gbar;
+  unsigned* gen = gbar + 1;
+  const unsigned g0 = ld_acquire_gpu(gen);
+  __threadfence();
+  if (atomicAdd(count, 1u) == ctas - 1) {
+    atomicExch(count, 0u);
+    __threadfence();
+    st_release_gpu(gen, g0 + 1);
+    return true;
+  }
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_gpu(gen) == g0) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, kStatusTimeout);
+      atomicExch(&g_wait_site, 30u);
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+template <int KIND>
+__device__ __forceinline__ void fused_act_quant(const GemmParams& p, volatile int* abort) {
+  constexpr int kWarps = KindTraits<KIND>::kThreads / 32;
+  const unsigned ctas = gridDim.x * gridDim.y;
+  const unsigned b = blockIdx.y * gridDim.x + blockIdx.x;
+  const int rb0 = static_cast<int>(static_cast<int64_t>(p.M) * b / ctas);
+  const int rb1 = static_cast<int>(static_cast<int64_t>(p.M) * (b + 1) / ctas);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = p.K >> 3;  // 16-byte chunks per row
+  for (int r = rb0 + warp; r < rb1; r += kWarps) {
+    const uint4* xr = reinterpret_cast<const uint4*>(p.xf16 + static_cast<int64_t>(r) * p.K);
+    float a = 0.0f;
+    for (int c = lane; c < nch; c += 32) a = fmaxf(a, absmax8(__ldg(xr + c)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const float s = __fdiv_rn(a, 127.0f);
+    uint2* qr = reinterpret_cast<uint2*>(p.xq_ws + static_cast<int64_t>(r) * p.K);
+    for (int c = lane; c < nch; c += 32) qr[c] = quant8_i8(__ldg(xr + c), s, a == 0.0f);
+    if (lane == 0) p.sx_ws[r] = s;
+  }
+  // the codes are read by other CTAs' TMA loads (async proxy)
+  __threadfence();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0) grid_barrier(p.gbar, ctas, abort);
+  __syncthreads();
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ kernel --
 template <int KIND>
 __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
@@ -564,6 +649,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   if (threadIdx.x == 0) ARIA_STAMP(1);
   pdl_wait();
   pdl_launch_dependents();
+  if constexpr (KIND == kW8A8) {
+    if (p.xf16) fused_act_quant<KIND>(p, abort_flag);
+  }
   if (threadIdx.x == 0) ARIA_STAMP(2);
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
 

@@ -285,3 +285,41 @@ def test_steer_schedule_window():
     assert aq.steer_schedule("residual:12:v:0.3:0-7", 8) == [0.3] * 8
     assert aq.steer_schedule("residual:12:v:0.5:2-4", 8) == [0, 0, 0.5, 0.5, 0.5, 0, 0, 0]
     assert aq.steer_schedule("residual:12:v:0.5:6-9", 8) == [0] * 6 + [0.5, 0.5]   # clipped to the run
+
+
+# ------------------------------------------------- fused W8A8 workspace ---
+
+def test_w8a8_workspace_size(lib):
+    assert aq.w8a8_workspace_size(432, 1536) == 256 + 1792 + 432 * 1536      # 4*432 -> 1792
+    assert aq.w8a8_workspace_size(1, 16) == 256 + 256 + 16
+    with pytest.raises(aq.AriaError):
+        aq.w8a8_workspace_size(0, 16)
+
+
+def test_fused_w8a8_rules(lib):
+    P = ctypes.c_void_p
+    need = aq.w8a8_workspace_size(4, 16)
+    ws = P(0x20000)
+    f = lib.aria_qgemm_w8a8_fused
+    # NULL workspace, too small a workspace, misaligned workspace
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, None, need, None) == 1
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, ws, need - 1, None) == 1
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, P(0x20010), need, None) == 3
+    # shape rules as for the W8A8 GEMM
+    assert f(4, 24, 16, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, ws, need, None) == 2
+    k_bad = (KMAX_I8 // 16 + 1) * 16
+    big = aq.w8a8_workspace_size(4, k_bad)
+    assert f(4, 16, k_bad, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, ws, big, None) == 2
+    # a misaligned device alpha
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, None, OK_PTR, 0.0, P(0x10002), OK_PTR, ws, need,
+             None) == 3
+
+
+def test_workspace_codes_layout():
+    import torch
+    M, K = 5, 32
+    ws = torch.arange(aq.w8a8_workspace_size(M, K), dtype=torch.int64).to(torch.uint8)
+    xq, sx = aq.workspace_codes(ws, M, K)
+    assert xq.shape == (M, K) and sx.shape == (M,)
+    assert xq.view(torch.uint8)[0, 0].item() == (256 + 256) % 256           # codes after 256 + 256
+    assert sx.view(torch.uint8).flatten()[0].item() == 256 % 256

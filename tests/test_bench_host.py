@@ -130,3 +130,14 @@ def test_fp16_rung_account():
     assert acc["f16"][0] == acc["q8"][0]
     xy = sum(2 * 432 * k + 2 * 432 * n for _, k, n in bench.LINEARS)
     assert acc["f16"][1] == 8 * (24 * (2 * params + xy) + 4 * 1536)
+
+
+def test_fused_w8a8_account():
+    """The fused W8A8 leg counts the fp16 activations once, not the codes'
+    round trip through the workspace."""
+    acc = bench.step_account()
+    assert acc["w8a8"][0] == acc["q8"][0]
+    params = 1536 * 4608 + 1536 * 1536 + 1536 * 6144 + 6144 * 1536
+    per_block = params + sum(2 * 432 * k + 4 * n + 2 * 432 * n for _, k, n in bench.LINEARS)
+    assert acc["w8a8"][1] == 8 * (24 * per_block + 4 * 1536)
+    assert bench.Replay.ORDER == ("q8", "w8a8", "q4")

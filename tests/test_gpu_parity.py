@@ -514,6 +514,7 @@ def test_bench_replay_outputs_match_oracle():
         for kind in kinds:
             for key in rep.y.get(kind.replace("_gemm", ""), {}):
                 rep.y[kind.replace("_gemm", "")][key].fill_(float("nan"))   # no stale result passes
+        torch.cuda.synchronize()
         with torch.cuda.stream(rep.stream):
             for kind in kinds:
                 rep.graphs[kind, buf if kind != "w8a8_gemm" else 0].replay()
@@ -528,14 +529,16 @@ def test_bench_replay_outputs_match_oracle():
                 vv, a = steer(b, name)
                 check_wo(f16np(rep.y["q8"][b, name])[rows],
                          oracle.wo_ref("q8", x, Wq, sw, None, vv, a, rows=rows))
-        replay(buf, "act_quant", "w8a8_gemm")
-        for b in blocks:
-            for name, k, n in bench.LINEARS:
-                x = rep.x_host[b, name].numpy()
-                Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
-                vv, a = steer(b, name)
-                ref = oracle.w8a8(x, Wq, sw, None, vv, a, rows=rows)
-                assert np.array_equal(f16np(rep.y["w8a8"][b, name]).view(np.uint16)[rows], ref), (b, name)
+        for w8a8_kinds in (("w8a8",), ("act_quant", "w8a8_gemm")):   # fused, and separate launches
+            replay(buf, *w8a8_kinds)
+            for b in blocks:
+                for name, k, n in bench.LINEARS:
+                    x = rep.x_host[b, name].numpy()
+                    Wq, sw = (t.cpu().numpy() for t in rep.q8[b, name])
+                    vv, a = steer(b, name)
+                    ref = oracle.w8a8(x, Wq, sw, None, vv, a, rows=rows)
+                    assert np.array_equal(f16np(rep.y["w8a8"][b, name]).view(np.uint16)[rows], ref), \
+                        (w8a8_kinds, b, name)
         replay(buf, "q4")
         for b in blocks:
             for name, k, n in bench.LINEARS:
