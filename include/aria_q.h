@@ -228,6 +228,25 @@ aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t *Xq, co
                            int32_t *C, void *stream);
 
 /*
+ * aria_selftest_bounded_wait -- failure-detection self-test (no counterpart
+ * on the pages; the library's own fault path). Launches the W8A8 GEMM of
+ * aria_qgemm(ARIA_FMT_W8A8) with every bounded wait limited to
+ * wait_limit_us microseconds and with the first pipeline stage of each
+ * CTA's first tile withheld, so that the waits on that stage run out. The
+ * kernel then unwinds without hanging or faulting: the waiting roles give
+ * up, the copies already in flight are drained, tensor memory is freed, and
+ * the device status word records the timeout. aria_device_status() on the
+ * same stream then returns ARIA_ERR_TIMEOUT (and clears it); Y is left
+ * unspecified; the context stays usable for the next call.
+ *   Xq, sx, Wq, sw, Y  as for aria_qgemm(ARIA_FMT_W8A8) (device, 16-byte aligned).
+ *   wait_limit_us      1 .. 4000000 (INVALID_ARG otherwise).
+ * Shape rules as for aria_qgemm(ARIA_FMT_W8A8).
+ */
+aria_status aria_selftest_bounded_wait(int64_t M, int64_t N, int64_t K, const int8_t *Xq,
+                                       const float *sx, const int8_t *Wq, const float *sw,
+                                       void *Y, uint32_t wait_limit_us, void *stream);
+
+/*
  * aria_device_status -- synchronise `stream`, then read and clear the device
  * status word of the current device. Returns ARIA_ERR_TIMEOUT if any kernel
  * of this library gave up on a bounded wait since the last call, ARIA_ERR_CUDA

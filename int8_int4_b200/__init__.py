@@ -31,7 +31,7 @@ STATUS = {0: "ARIA_OK", 1: "ARIA_ERR_INVALID_ARG", 2: "ARIA_ERR_UNSUPPORTED",
 FORMATS = {"q8": 1, "q4": 2, "w8a8": 3, "f16": 4}
 API = ("aria_status_string", "aria_last_error_message", "aria_qpack_size", "aria_qpack",
        "aria_act_quant", "aria_qgemm", "aria_qgemm_steer_dev", "aria_w8a8_workspace_size",
-       "aria_qgemm_w8a8_fused", "aria_qgemm_s32", "aria_device_status")
+       "aria_qgemm_w8a8_fused", "aria_qgemm_s32", "aria_selftest_bounded_wait", "aria_device_status")
 
 
 class AriaError(RuntimeError):
@@ -64,6 +64,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "aria_qgemm_w8a8_fused": ([I64, I64, I64, P, P, P, P, P, ctypes.c_float, P, P, P,
                                    ctypes.c_size_t, P], I),
         "aria_qgemm_s32": ([I64, I64, I64, P, P, P, P], I),
+        "aria_selftest_bounded_wait": ([I64, I64, I64, P, P, P, P, P, ctypes.c_uint32, P], I),
         "aria_device_status": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -327,6 +328,26 @@ def qgemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out=None, stream=None):
                                              _dev(Wq, "Wq", torch.int8), _dev(C, "out", torch.int32),
                                              _stream(stream)))
     return C
+
+
+def selftest_bounded_wait(Xq, sx, Wq, sw, out=None, wait_limit_us: int = 50000, stream=None):
+    """Failure-detection self-test (include/aria_q.h): a W8A8 launch whose
+    first pipeline stage never fills, with every bounded wait limited to
+    wait_limit_us. Returns the output tensor (contents unspecified); the
+    following device_status() raises AriaError with ARIA_ERR_TIMEOUT."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    _expect(sx, "sx", (M,), torch.float32)
+    _expect(Wq, "Wq", (N, K), torch.int8)
+    _expect(sw, "scales", (N,), torch.float32)
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=Xq.device)
+    _expect(Y, "out", (M, N), torch.float16)
+    same_device(Xq=Xq, sx=sx, Wq=Wq, sw=sw, out=Y)
+    with _on(Xq.device):
+        _check(load_library().aria_selftest_bounded_wait(
+            M, N, K, _dev(Xq, "Xq", torch.int8), _dev(sx, "sx", torch.float32), _dev(Wq, "Wq", torch.int8),
+            _dev(sw, "scales", torch.float32), _dev(Y, "out"), int(wait_limit_us), _stream(stream)))
+    return Y
 
 
 def device_status(stream=None):

@@ -620,11 +620,18 @@ FusedWs fused_ws(void* ws, int64_t M) {
                  reinterpret_cast<int8_t*>(b + kWsHeader + sx)};
 }
 
+// the failure-detection self-test's settings of a launch (defaults: none)
+struct SelfTest {
+  uint64_t wait_ns = 0;
+  int drop_first_stage = 0;
+};
+
 static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const void* X,
                               const float* sx, const void* Wq, const void* scales,
                               const void* bias, const float* steer, float alpha,
                               const float* alpha_dev, void* Y, cudaStream_t st,
-                              const void* xf16 = nullptr, const FusedWs* ws = nullptr) {
+                              const void* xf16 = nullptr, const FusedWs* ws = nullptr,
+                              const SelfTest& selftest = SelfTest{}) {
   using namespace aria;
   aria_status s = check_gemm_shape(M, N, K);
   if (s != ARIA_OK) return s;
@@ -635,7 +642,7 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
                 (long long)(INT32_MAX / (127 * 127)), (long long)K);
   // a handful of tokens: the weight-streaming kernel, when its plan fits
   SmallPlan sp;
-  if (!xf16 && plan_small(kind, M, N, K, &sp)) {
+  if (!xf16 && !selftest.drop_first_stage && plan_small(kind, M, N, K, &sp)) {
     sp.p.W = static_cast<const uint8_t*>(Wq);
     sp.p.Wsc = kind == kQ4 ? static_cast<const __half*>(scales) : nullptr;
     sp.p.sw = kind == kQ8 ? static_cast<const float*>(scales) : nullptr;
@@ -680,6 +687,8 @@ static aria_status qgemm_impl(int kind, int64_t M, int64_t N, int64_t K, const v
   pl.p.alpha = pl.p.steer ? alpha : 0.0f;
   pl.p.alpha_dev = pl.p.steer ? alpha_dev : nullptr;
   pl.p.Y = Y;
+  pl.p.wait_ns = selftest.wait_ns;
+  pl.p.drop_first_stage = selftest.drop_first_stage;
   if (xf16) {  // W8A8 with the activation quantisation in this launch
     pl.p.xf16 = static_cast<const __half*>(xf16);
     pl.p.xq_ws = ws->xq;
@@ -792,6 +801,23 @@ ARIA_API aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_
     return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
   return qgemm_impl(aria::kS32, M, N, K, Xq, nullptr, Wq, Wq, nullptr, nullptr, 0.0f, nullptr, C,
                     static_cast<cudaStream_t>(stream));
+}
+
+ARIA_API aria_status aria_selftest_bounded_wait(int64_t M, int64_t N, int64_t K, const int8_t* Xq,
+                                               const float* sx, const int8_t* Wq, const float* sw,
+                                               void* Y, uint32_t wait_limit_us, void* stream) {
+  if (!Xq || !sx || !Wq || !sw || !Y) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  for (const void* q : {static_cast<const void*>(Xq), static_cast<const void*>(sx),
+                        static_cast<const void*>(Wq), static_cast<const void*>(sw),
+                        static_cast<const void*>(Y)})
+    if (!aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  if (wait_limit_us < 1 || wait_limit_us > 4000000u)
+    return fail(ARIA_ERR_INVALID_ARG, "wait_limit_us must be in [1, 4e6]");
+  SelfTest t;
+  t.wait_ns = static_cast<uint64_t>(wait_limit_us) * 1000u;
+  t.drop_first_stage = 1;
+  return qgemm_impl(aria::kW8A8, M, N, K, Xq, sx, Wq, sw, nullptr, nullptr, 0.0f, nullptr, Y,
+                    static_cast<cudaStream_t>(stream), nullptr, nullptr, t);
 }
 
 ARIA_API aria_status aria_device_status(void* stream) {

@@ -82,17 +82,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete, or give up after
-// kWaitLimitNs, or as soon as another thread of the CTA has raised *abort.
+// `limit_ns`, or as soon as another thread of the CTA has raised *abort.
 // On giving up: records the site in the device status word, raises *abort
 // and returns false. The caller then stops its role and goes to teardown.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                       uint32_t site) {
+                                       uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(&g_status, kStatusTimeout);
       atomicExch(&g_wait_site, site);
       *abort = 1;
@@ -105,23 +105,24 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
 // already), the out-of-line bounded loop only when it has not. A call in the
 // issue loop of the MMA or TMA thread costs hundreds of cycles per stage.
 __device__ __forceinline__ bool mbar_wait_fast(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                               uint32_t site) {
+                                               uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait(bar, parity, abort, site);
+  return mbar_wait(bar, parity, abort, site, limit_ns);
 }
 
 // Warp-converged form for a role that runs as a whole warp: every lane waits,
 // and the result is made warp-uniform.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                               uint32_t site) {
-  return __all_sync(0xffffffffu, mbar_wait_fast(bar, parity, abort, site));
+                                               uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, mbar_wait_fast(bar, parity, abort, site, limit_ns));
 }
 
 // Same, ignoring the abort flag: used at teardown to drain copies in flight.
-__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                             uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       atomicOr(&g_status, kStatusTimeout);
       return false;
     }

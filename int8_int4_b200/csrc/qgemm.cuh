@@ -76,6 +76,11 @@ struct GemmParams {
   int8_t* xq_ws;
   float* sx_ws;
   unsigned* gbar;
+  // failure-detection self-test: the limit of every bounded wait (0: the
+  // default kWaitLimitNs) and, for W8A8 / fp16, a hook that withholds the
+  // first stage of each CTA's first tile so that the waits on it run out
+  uint64_t wait_ns;
+  int drop_first_stage;
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
@@ -534,6 +539,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint64_t wlim = p.wait_ns ? p.wait_ns : kWaitLimitNs;
+  const bool drop0 = !T::kDequant && p.drop_first_stage != 0;  // self-test hook
   if (threadIdx.x == 0) ARIA_STAMP(0);
   const bool split = p.splits > 1;
   const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
@@ -633,6 +640,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       pre = nkb < p.n_a ? nkb : p.n_a;
       if (lane == 0) {
         for (int i = 0; i < pre; ++i) {
+          if (i == 0 && drop0) continue;  // self-test: this stage never fills
           mbar_arrive_expect_tx(st_full + i, kATile + p.x_stage);
           tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * T::kWUnitX, n0, pol);
         }
@@ -673,7 +681,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             if (++s == p.n_raw) { s = 0; ph ^= 1u; }
             continue;
           }
-          if (!(ok = mbar_wait_warp(raw_empty + s, ph ^ 1, abort_flag, 1))) break;
+          if (!(ok = mbar_wait_warp(raw_empty + s, ph ^ 1, abort_flag, 1, wlim))) break;
           if (lane == 0) {
             uint8_t* dst = raw + s * p.raw_stage;
             const int u = u_begin + i;
@@ -700,13 +708,13 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           if (tile == tile0 && kb < pre) {
             // the weight half went out before the dependency wait (the barrier
             // already expects both halves): add the activation half
-            if (lane == 0)
+            if (lane == 0 && !(kb == 0 && drop0))
               tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (u_begin + kb) * T::kXElemsPerKb, m0,
                           polx);
             if (++s == p.n_a) { s = 0; ph ^= 1u; }
             continue;
           }
-          if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2))) break;
+          if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2, wlim))) break;
           if (lane == 0) {
             if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * T::kWUnitX, n0);
             mbar_arrive_expect_tx(st_full + s, kATile + p.x_stage);
@@ -729,7 +737,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
       const int m0 = (tile / p.tiles_n) * p.BN;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 3))) break;
+        if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 3, wlim))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(st_full + s, p.x_stage);
           tma_load_2d(&tmX, st_full + s, xbuf + s * p.x_stage, (kx0 + kb) * T::kXElemsPerKb, m0, pol);
@@ -746,12 +754,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     bool ok = true;
     for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
       const int b = ti & 1;
-      if (!(ok = mbar_wait_warp(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9))) break;
+      if (!(ok = mbar_wait_warp(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9, wlim))) break;
       if (ti == 0 && lane == 0) ARIA_STAMP(3);
       tc_fence_after();
       const uint32_t dt = tmem_base + b * kAccCols;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!(ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4))) break;
+        if (!(ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4, wlim))) break;
         if (kb == 0 && ti == 0 && lane == 0) ARIA_STAMP(4);
         tc_fence_after();
         const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
@@ -779,7 +787,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       bool ok = true;
       for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
         for (int i = 0; i < nu && ok; ++i) {
-          if (!(ok = mbar_wait_fast(raw_full + s, rph, abort_flag, 6))) break;
+          if (!(ok = mbar_wait_fast(raw_full + s, rph, abort_flag, 6, wlim))) break;
           if (t == 0 && tile == tile0 && i == 0) ARIA_STAMP(12);
           const uint8_t* src = raw + s * p.raw_stage;
           uint4 v[8];
@@ -797,7 +805,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           if (++s == p.n_raw) { s = 0; rph ^= 1u; }
 #pragma unroll
           for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
-            if (!(ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7))) break;
+            if (!(ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7, wlim))) break;
             uint8_t* dst = abuf + sa * kATile;
             if constexpr (KIND == kQ8) {
               // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
@@ -842,7 +850,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         const int n0 = (tile % p.tiles_n) * kTileN;
         const int m0 = (tile / p.tiles_n) * p.BN;
         const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
-        bool ok2 = mbar_wait(acc_last, 0, abort_flag, 10);
+        bool ok2 = mbar_wait(acc_last, 0, abort_flag, 10, wlim);
         ok2 = __all_sync(0xffffffffu, ok2);
         if (ok2) {
           tc_fence_after();
@@ -881,7 +889,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           for (int j = te; j < p.BN; j += nep) sxs[j] = (m0 + j < p.M) ? __ldg(p.sx + m0 + j) : 0.0f;
           named_bar(1, nep);
         }
-        bool ok = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 8);
+        bool ok = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 8, wlim);
         ok = __all_sync(0xffffffffu, ok);  // warp-uniform before .sync.aligned TMEM loads
         if (!ok) continue;  // keep taking part in the named barriers of later tiles
         if (te == 0 && ti == 0) ARIA_STAMP(6);
@@ -923,7 +931,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   // once, then sums them in rank order (deterministic) and applies the
   // epilogue.
   if (split) {
-    epi_ok = mbar_wait_warp(acc_full, 0, abort_flag, 8);
+    epi_ok = mbar_wait_warp(acc_full, 0, abort_flag, 8, wlim);
     const int lg = warp & 3, wg = warp >> 2;  // TMEM lane group; third of the columns
     uint32_t* red = reinterpret_cast<uint32_t*>(smem);
     {
@@ -1050,7 +1058,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       const int nring = T::kDequant ? p.n_raw : p.n_a;
       uint64_t* full = T::kDequant ? raw_full : st_full;
       for (int i = (issued_w > nring ? issued_w - nring : 0); i < issued_w; ++i)
-        mbar_wait_drain(full + (i % nring), (i / nring) & 1);
+        if (!(i == 0 && drop0))  // a withheld stage has nothing in flight
+          mbar_wait_drain(full + (i % nring), (i / nring) & 1, wlim);
     } else if (warp == 2 && issued_x > 0) {
       const uint64_t t0 = globaltimer();  // X loads of q8/q4: allow 100 us to land
       while (globaltimer() - t0 < 100000ull) __nanosleep(1000);
@@ -1060,7 +1069,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     // MMAs issued before the abort finish before TMEM is freed; the commit
     // comes from the lane that issued them (elect.sync, as in the issue loop)
     umma_commit_elect(mma_drain);
-    mbar_wait_drain(mma_drain, 0);
+    mbar_wait_drain(mma_drain, 0, wlim);
   }
   tc_fence_before();
   __syncthreads();

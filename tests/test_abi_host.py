@@ -323,3 +323,12 @@ def test_workspace_codes_layout():
     assert xq.shape == (M, K) and sx.shape == (M,)
     assert xq.view(torch.uint8)[0, 0].item() == (256 + 256) % 256           # codes after 256 + 256
     assert sx.view(torch.uint8).flatten()[0].item() == 256 % 256
+
+
+def test_selftest_rules(lib):
+    f = lib.aria_selftest_bounded_wait
+    assert f(4, 16, 16, None, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 1000, None) == 1
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 0, None) == 1          # limit 0
+    assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 4000001, None) == 1    # above 4 s
+    assert f(4, 16, 16, OK_PTR, OK_PTR, ctypes.c_void_p(0x10008), OK_PTR, OK_PTR, 1000, None) == 3
+    assert f(4, 24, 16, OK_PTR, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 1000, None) == 2       # N % 16
