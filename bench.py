@@ -12,12 +12,11 @@ denoising loop replayed as one CUDA graph; "Live steering while streaming":
 the steering strength lives inside the captured graph, here a device-side
 schedule read by the steered launch of each step). Weights are packed once
 at load, as on the pages. Per precision one CUDA graph holds the 8-step loop
-(768 GEMM launches; the W8A8 launches quantise their activations per token
-inside the same kernel).
+(768 GEMM launches; W8A8 adds 768 per-token activation quantisations).
 
 Beside the step, outside `value`: the unquantised fp16 rung of the
-precision ladder on the same replay, the W8A8 leg with a separate
-activation-quantisation launch before each GEMM, the steering on/off delta (the same
+precision ladder on the same replay, the W8A8 leg with the activation
+quantisation fused into the GEMM launch, the steering on/off delta (the same
 graphs with the schedule set to 0), every per-shape case of the benchmark
 configurations (`per_config`: q8 d=1024 at M in {1,16,432}, W8A8 d=1536 at
 M in {432,4096} with its activation quantisation, q4 d=1536 at M in
@@ -300,8 +299,8 @@ class Replay:
     step's inputs while the current step computes. The steered launch of
     step s reads its strength from `alpha[s]` (device memory)."""
 
-    ORDER = ("q8", "w8a8", "q4")                          # the timed step
-    EXTRA = ("act_quant", "w8a8_gemm", "f16")             # timed beside it
+    ORDER = ("q8", "act_quant", "w8a8_gemm", "q4")        # the timed step
+    EXTRA = ("w8a8_fused", "f16")                         # timed beside it
     LAUNCHES_PER_STEP = len(ORDER) * STEPS * BLOCKS * len(LINEARS)
 
     def __init__(self, dev, buffers=1, fp16=True):
@@ -361,7 +360,7 @@ class Replay:
                     elif kind == "f16":
                         aq.qgemm("f16", x[key], self.w16[key], None, out=self.y["f16"][key],
                                  stream=stream, **self._steer(s, b, name))
-                    elif kind == "w8a8":
+                    elif kind == "w8a8_fused":
                         aq.qgemm_w8a8_fused(x[key], *self.q8[key], out=self.y["w8a8"][key],
                                             workspace=self.ws, stream=stream, **self._steer(s, b, name))
                     elif kind == "act_quant":
@@ -488,10 +487,10 @@ def run_ours(args, ws, rank):
     rep.alpha.zero_()
     off_ms, _ = time_steps(rep, args.steps, ws)
     rep.alpha.fill_(synthetic.REPLAY_ALPHA)
-    # the W8A8 leg with a separate activation-quantisation launch (outside `value`)
+    # the W8A8 leg with the activation quantisation fused into the GEMM launch (outside `value`)
     for _ in range(max(1, args.warmup // 2)):
-        rep.run_step(kinds=("act_quant", "w8a8_gemm"))
-    unf_ms, unf_seg = time_steps(rep, args.steps, ws, kinds=("act_quant", "w8a8_gemm"))
+        rep.run_step(kinds=("w8a8_fused",))
+    fus_ms, _ = time_steps(rep, args.steps, ws, kinds=("w8a8_fused",))
     # the fp16 rung of the precision ladder, same replay (outside `value`)
     f16_ms = None
     if rep.fp16:
@@ -510,16 +509,16 @@ def run_ours(args, ws, rank):
     barrier(ws)
     rep.aq.device_status(rep.stream)
 
-    vals = max_over_ranks([total_ms, e2e_ms, off_ms, f16_ms or 0.0, unf_ms, *unf_seg, *seg_ms], ws)
-    total_ms, e2e_ms, off_ms, f16_ms_max, unf_ms, aq_ms, g_ms, *seg_ms = vals
+    vals = max_over_ranks([total_ms, e2e_ms, off_ms, f16_ms or 0.0, fus_ms, *seg_ms], ws)
+    total_ms, e2e_ms, off_ms, f16_ms_max, fus_ms, *seg_ms = vals
     if f16_ms is not None:
         f16_ms = f16_ms_max
 
-    ops_step = acct["q8"][0] + acct["q4"][0] + acct["w8a8"][0]
+    ops_step = acct["q8"][0] + acct["q4"][0] + acct["w8a8_gemm"][0]
     ms_per_step = total_ms / args.steps
     value = ops_step * ws / (ms_per_step * 1e-3) / 1e12
     hbm = R["hbm"]
-    kinds = {"q8": (0, R["f16"]), "w8a8": (1, R["i8"]), "q4": (2, R["f16"])}
+    kinds = {"q8": (0, R["f16"]), "act_quant": (1, None), "w8a8_gemm": (2, R["i8"]), "q4": (3, R["f16"])}
     launches = STEPS * BLOCKS * len(LINEARS)
     per = {}
     for kind, (i, peak) in kinds.items():
@@ -529,17 +528,18 @@ def run_ours(args, ws, rank):
         d.update(ms_per_step=seg_ms[i] / args.steps, launches_per_step=launches,
                  avg_launch_us=t / launches * 1e6)
         per[kind] = d
-    per["w8a8"]["note"] = ("activation quantisation inside the GEMM launch "
-                           "(aria_qgemm_w8a8_fused); algorithmic bytes: fp16 X, packed weights and "
-                           "scales, fp16 Y")
-    unfused = {"ms_per_step": unf_ms / args.steps,
-               "act_quant_ms_per_step": aq_ms / args.steps, "gemm_ms_per_step": g_ms / args.steps,
-               "act_quant": roof_entry(0.0, acct["act_quant"][1], aq_ms / args.steps * 1e-3, 1.0, hbm),
-               "gemm": roof_entry(acct["w8a8_gemm"][0], acct["w8a8_gemm"][1], g_ms / args.steps * 1e-3,
-                                  R["i8"], hbm),
-               "note": "the same W8A8 leg with a separate aria_act_quant launch before each "
-                       "aria_qgemm(W8A8): 1536 launches per step instead of 768"}
-    per_precision = {"q8": per["q8"], "q4": per["q4"], "w8a8": dict(per["w8a8"], unfused=unfused)}
+    fused = roof_entry(acct["w8a8"][0], acct["w8a8"][1], fus_ms / args.steps * 1e-3, R["i8"], hbm)
+    fused.update(ms_per_step=fus_ms / args.steps, launches_per_step=launches,
+                 avg_launch_us=fus_ms / args.steps * 1e-3 / launches * 1e6,
+                 note="the same W8A8 leg with the activation quantisation inside the GEMM launch "
+                      "(aria_qgemm_w8a8_fused, 768 launches per step instead of 1536); algorithmic "
+                      "bytes: fp16 X, packed weights and scales, fp16 Y; timed after the step, not in value")
+    t_w = (seg_ms[1] + seg_ms[2]) / args.steps
+    per_precision = {
+        "q8": per["q8"], "q4": per["q4"],
+        "w8a8": {"ms_per_step": t_w, "tops": acct["w8a8_gemm"][0] / (t_w * 1e-3) / 1e12,
+                 "gemm": per["w8a8_gemm"], "act_quant": per["act_quant"], "fused": fused},
+    }
     if f16_ms is not None:
         t = f16_ms / args.steps * 1e-3
         d = roof_entry(acct["f16"][0], acct["f16"][1], t, R["f16"], hbm)
@@ -554,19 +554,20 @@ def run_ours(args, ws, rank):
     t_l = dd["avg_launch_us"] * 1e-6
     if dd["bound"] == "tensor":
         roof = {"bound": "tensor", "achieved": ops_l / t_l / 1e12, "peak": kinds[dom][1],
-                "unit": "TFLOP/s" if dom != "w8a8" else "TOPS"}
+                "unit": "TFLOP/s" if dom != "w8a8_gemm" else "TOPS"}
     else:
         roof = {"bound": "hbm", "achieved": byt_l / t_l / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = {"q8": "qgemm_kernel<Q8>", "q4": "qgemm_kernel<Q4>", "w8a8": "qgemm_kernel<W8A8>"}[dom]
+    roof["kernel"] = {"q8": "qgemm_kernel<Q8>", "q4": "qgemm_kernel<Q4>", "w8a8_gemm": "qgemm_kernel<W8A8>",
+                      "act_quant": "row_quant_i8_kernel"}[dom]
     roof["traffic"], roof["traffic_source"] = measured_traffic(roof["kernel"], acct[dom][1] / launches)
     roof["peak_source"] = (f"{peak_src} MEASURED_PEAKS.json "
                            + ("bf16_tflops (burst: the kernel runs inside a ~30 ms step at full clocks)"
                               if roof["bound"] == "tensor" else "hbm_gbs")
-                           + (" x 2 (nominal int8:fp16)" if dom == "w8a8" else ""))
+                           + (" x 2 (nominal int8:fp16)" if dom == "w8a8_gemm" else ""))
     if roof["bound"] == "tensor":
         roof["frac_of_sustained"] = roof["achieved"] / (
-            peaks["bf16_tflops_sustained"] * (INT8_OVER_F16 if dom == "w8a8" else 1.0))
+            peaks["bf16_tflops_sustained"] * (INT8_OVER_F16 if dom == "w8a8_gemm" else 1.0))
     roof["per_launch"] = {"ops": ops_l, "bytes": byt_l, "avg_us": t_l * 1e6}
 
     line = {

@@ -198,16 +198,18 @@ aria_status aria_w8a8_workspace_size(int64_t M, int64_t K, size_t *bytes);
  *              followed by aria_qgemm(ARIA_FMT_W8A8).
  *   workspace  caller-owned device memory, 256-byte aligned, at least
  *              aria_w8a8_workspace_size(M, K) bytes (INVALID_ARG otherwise).
- *              Its first 256 bytes hold a grid barrier and must be zero
- *              before the first call; every successful call leaves them
- *              zero. After the call the workspace holds the token scales
+ *              Its first 256 bytes hold a grid barrier: bytes 0..3 (the
+ *              arrival count) must be zero before the first call, and every
+ *              successful call leaves them zero; bytes 4..7 count the calls
+ *              (any starting value). After the call the workspace holds the
+ *              token scales
  *              (fp32 [M] at byte 256) and the codes (int8 [M,K] at byte
  *              256 + 4*M rounded up to 256), as aria_act_quant would write
  *              them. Calls that share a workspace must not overlap on the
  *              GPU (one stream, or ordered by events).
  *   The kernel's CTAs meet at a grid-wide barrier after quantising their
  *   share of the rows; its wait is bounded: if it runs out, the device
- *   status word reports ARIA_ERR_TIMEOUT and the workspace's first 256 bytes
+ *   status word reports ARIA_ERR_TIMEOUT and the workspace's arrival count
  *   must be zeroed again before the next call.
  * Shape rules and stream order as for aria_qgemm(ARIA_FMT_W8A8).
  */

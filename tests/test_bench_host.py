@@ -140,4 +140,5 @@ def test_fused_w8a8_account():
     params = 1536 * 4608 + 1536 * 1536 + 1536 * 6144 + 6144 * 1536
     per_block = params + sum(2 * 432 * k + 4 * n + 2 * 432 * n for _, k, n in bench.LINEARS)
     assert acc["w8a8"][1] == 8 * (24 * per_block + 4 * 1536)
-    assert bench.Replay.ORDER == ("q8", "w8a8", "q4")
+    assert bench.Replay.ORDER == ("q8", "act_quant", "w8a8_gemm", "q4")
+    assert "w8a8_fused" in bench.Replay.EXTRA

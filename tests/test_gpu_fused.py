@@ -8,7 +8,8 @@ the rows, then a grid-wide barrier) instead of in a separate launch. Its
 output must be the same bytes as aria_act_quant followed by
 aria_qgemm(W8A8); the codes and token scales it leaves in its workspace must
 equal the oracle's bit for bit; the grid barrier must leave the workspace
-ready for the next call (its header back to zero).
+ready for the next call (its arrival count back to zero; the generation
+word counts the calls).
 """
 import numpy as np
 import pytest
@@ -65,7 +66,7 @@ def test_fused_equals_separate_and_oracle(M, N, K, epi):
     rq, rs = oracle.act_quant(X.numpy())
     assert np.array_equal(wq.cpu().numpy(), rq)
     assert np.array_equal(wsx.cpu().numpy().view(np.uint32), rs.view(np.uint32))
-    assert not ws[:256].any(), "grid barrier header not reset"
+    assert not ws[:4].any(), "grid barrier arrival count not reset"
     rows = sample_rows(M, 16)
     ref = oracle.w8a8(X.numpy(), Wq.cpu().numpy(), sw.cpu().numpy(), None if b is None else b.numpy(),
                       None if v is None else v.numpy(), alpha, rows=rows)
@@ -90,7 +91,8 @@ def test_fused_repeated_calls_and_device_alpha():
     dev0 = aq.qgemm_w8a8_fused(Xd, Wq, sw, steer_vec=v, alpha_dev=sched[1:2], workspace=ws)
     assert torch.equal(dev0.view(torch.int16), unsteered.view(torch.int16))
     torch.cuda.synchronize()
-    assert not ws[:256].any()
+    assert not ws[:4].any()                           # arrival count back to zero
+    assert ws[4:8].view(torch.int32).item() == 14     # the generation counts the calls
     aq.device_status()
 
 
@@ -151,6 +153,6 @@ def test_fused_in_a_dependent_chain(graph):
         y = h3[rows].astype(np.float64)
         ref3 = oracle.wo_ref("q4", h2, w3, sw3, rows=rows)
         assert np.abs(y - ref3).max() <= 1e-2 * np.abs(ref3).max()
-    assert not ws[:256].any()
+    assert not ws[:4].any()
     del g
     aq.device_status()

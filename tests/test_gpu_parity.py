@@ -512,8 +512,9 @@ def test_bench_replay_outputs_match_oracle():
 
     def replay(buf, *kinds):
         for kind in kinds:
-            for key in rep.y.get(kind.replace("_gemm", ""), {}):
-                rep.y[kind.replace("_gemm", "")][key].fill_(float("nan"))   # no stale result passes
+            prec = kind.replace("_gemm", "").replace("_fused", "")
+            for key in rep.y.get(prec, {}):
+                rep.y[prec][key].fill_(float("nan"))   # no stale result passes
         torch.cuda.synchronize()
         with torch.cuda.stream(rep.stream):
             for kind in kinds:
@@ -529,7 +530,7 @@ def test_bench_replay_outputs_match_oracle():
                 vv, a = steer(b, name)
                 check_wo(f16np(rep.y["q8"][b, name])[rows],
                          oracle.wo_ref("q8", x, Wq, sw, None, vv, a, rows=rows))
-        for w8a8_kinds in (("w8a8",), ("act_quant", "w8a8_gemm")):   # fused, and separate launches
+        for w8a8_kinds in (("w8a8_fused",), ("act_quant", "w8a8_gemm")):   # fused, and separate launches
             replay(buf, *w8a8_kinds)
             for b in blocks:
                 for name, k, n in bench.LINEARS:
