@@ -219,6 +219,36 @@ aria_status aria_qgemm_w8a8_fused(int64_t M, int64_t N, int64_t K, const void *X
                                   size_t workspace_bytes, void *stream);
 
 /*
+ * aria_qgemm_w8a8_fused_noalloc -- aria_qgemm_w8a8_fused without a caller
+ * workspace and without allocating anything. The paper has no counterpart:
+ * this entry point exists for callers that must not allocate device memory
+ * while they run -- a real-time audio render callback, where cudaMalloc can
+ * block or synchronise the device and miss the deadline, or a host that
+ * fixes the device memory budget at load time and forbids allocation
+ * afterwards. Its scratch (the codes, the token scales and the grid barrier)
+ * is a static device array of ARIA_NOALLOC_SCRATCH_BYTES (32 MiB) inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.
+ *   Arguments and result as for aria_qgemm_w8a8_fused (no workspace).
+ *   Size limit: 256 + 4*M rounded up to 256 + M*K must not exceed
+ *   ARIA_NOALLOC_SCRATCH_BYTES; larger calls return ARIA_ERR_UNSUPPORTED and
+ *   launch nothing (e.g. M = 4096 allows K up to 8176).
+ *   The first call on a device looks up the scratch's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.
+ *   Each call clears the scratch's barrier words on `stream` before its
+ *   kernel (no allocation: a memset). All calls share the one scratch array,
+ *   which keeps the last call's contents: calls that overlap on the GPU
+ *   (different streams without ordering) race and give wrong results.
+ *   Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define ARIA_NOALLOC_SCRATCH_BYTES (32u << 20)
+aria_status aria_qgemm_w8a8_fused_noalloc(int64_t M, int64_t N, int64_t K, const void *X,
+                                          const void *Wq, const float *sw, const void *bias,
+                                          const float *steer_vec, float alpha, const float *alpha_dev,
+                                          void *Y, void *stream);
+
+/*
  * aria_qgemm_s32 -- the W8A8 integer GEMM alone: C[m,n] = sum_k Xq[m,k]*Wq[n,k]
  * as exact int32 ("Results": 8-bit arithmetic on integer tensor cores). Runs
  * the same tensor-core mainloop as aria_qgemm(ARIA_FMT_W8A8) and stores the

@@ -31,7 +31,8 @@ STATUS = {0: "ARIA_OK", 1: "ARIA_ERR_INVALID_ARG", 2: "ARIA_ERR_UNSUPPORTED",
 FORMATS = {"q8": 1, "q4": 2, "w8a8": 3, "f16": 4}
 API = ("aria_status_string", "aria_last_error_message", "aria_qpack_size", "aria_qpack",
        "aria_act_quant", "aria_qgemm", "aria_qgemm_steer_dev", "aria_w8a8_workspace_size",
-       "aria_qgemm_w8a8_fused", "aria_qgemm_s32", "aria_selftest_bounded_wait", "aria_device_status")
+       "aria_qgemm_w8a8_fused", "aria_qgemm_w8a8_fused_noalloc", "aria_qgemm_s32",
+       "aria_selftest_bounded_wait", "aria_device_status")
 
 
 class AriaError(RuntimeError):
@@ -63,6 +64,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "aria_w8a8_workspace_size": ([I64, I64, P], I),
         "aria_qgemm_w8a8_fused": ([I64, I64, I64, P, P, P, P, P, ctypes.c_float, P, P, P,
                                    ctypes.c_size_t, P], I),
+        "aria_qgemm_w8a8_fused_noalloc": ([I64, I64, I64, P, P, P, P, P, ctypes.c_float, P, P, P], I),
         "aria_qgemm_s32": ([I64, I64, I64, P, P, P, P], I),
         "aria_selftest_bounded_wait": ([I64, I64, I64, P, P, P, P, P, ctypes.c_uint32, P], I),
         "aria_device_status": ([P], I),
@@ -313,6 +315,34 @@ def qgemm_w8a8_fused(X: torch.Tensor, Wq: torch.Tensor, sw: torch.Tensor, bias=N
             float(alpha), None if alpha_dev is None else _dev(alpha_dev, "alpha_dev"),
             _dev(Y, "out"), _dev(workspace, "workspace"), workspace.numel(), _stream(stream)))
     return Y
+
+
+def qgemm_w8a8_fused_noalloc(X: torch.Tensor, Wq: torch.Tensor, sw: torch.Tensor, bias=None,
+                             steer_vec=None, alpha: float = 0.0, alpha_dev=None, out=None, stream=None):
+    """qgemm_w8a8_fused with the library's static scratch instead of a
+    workspace, for callers that must not allocate device memory while they
+    run (include/aria_q.h, aria_qgemm_w8a8_fused_noalloc). ``out`` must be
+    given: this call allocates nothing, not even its output."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    if out is None:
+        raise ValueError("qgemm_w8a8_fused_noalloc allocates nothing: pass out=")
+    _expect(X, "X", (M, K), torch.float16)
+    _expect(Wq, "Wq", (N, K), torch.int8)
+    _expect(sw, "scales", (N,), torch.float32)
+    _expect(bias, "bias", (N,), torch.float16)
+    _expect(steer_vec, "steer_vec", (N,), torch.float32)
+    _expect(out, "out", (M, N), torch.float16)
+    if alpha_dev is not None and (alpha_dev.numel() != 1 or alpha_dev.dtype != torch.float32):
+        raise TypeError("alpha_dev must be one float32 element")
+    same_device(X=X, Wq=Wq, scales=sw, bias=bias, steer_vec=steer_vec, out=out, alpha_dev=alpha_dev)
+    with _on(X.device):
+        _check(load_library().aria_qgemm_w8a8_fused_noalloc(
+            M, N, K, _dev(X, "X", torch.float16), _dev(Wq, "Wq", torch.int8), _dev(sw, "scales"),
+            _dev(bias, "bias", torch.float16), _dev(steer_vec, "steer_vec", torch.float32),
+            float(alpha), None if alpha_dev is None else _dev(alpha_dev, "alpha_dev"),
+            _dev(out, "out"), _stream(stream)))
+    return out
 
 
 def qgemm_s32(Xq: torch.Tensor, Wq: torch.Tensor, out=None, stream=None):

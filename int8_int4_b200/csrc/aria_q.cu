@@ -794,6 +794,60 @@ ARIA_API aria_status aria_qgemm_w8a8_fused(int64_t M, int64_t N, int64_t K, cons
                     static_cast<cudaStream_t>(stream), X, &ws);
 }
 
+// ------------------------------------------------- no-allocation variant ---
+// Scratch of aria_qgemm_w8a8_fused_noalloc: a file-scope device array that
+// every GPU loading this library holds until the process exits. Host code
+// must not pass the symbol itself to a kernel (on the host it names a
+// stand-in, not device memory): its device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = size_t{32} << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static aria_status noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return fail(ARIA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return ARIA_OK;
+}
+
+ARIA_API aria_status aria_qgemm_w8a8_fused_noalloc(int64_t M, int64_t N, int64_t K, const void* X,
+                                                   const void* Wq, const float* sw, const void* bias,
+                                                   const float* steer_vec, float alpha,
+                                                   const float* alpha_dev, void* Y, void* stream) {
+  if (!X || !Wq || !sw || !Y) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");
+  for (const void* q : {X, static_cast<const void*>(Wq), static_cast<const void*>(sw), bias,
+                        static_cast<const void*>(steer_vec), static_cast<const void*>(Y)})
+    if (q && !aligned16(q)) return fail(ARIA_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+  if (alpha_dev && (reinterpret_cast<uintptr_t>(alpha_dev) & 3u))
+    return fail(ARIA_ERR_MISALIGNED, "alpha_dev must be 4-byte aligned");
+  aria_status s = check_gemm_shape(M, N, K);
+  if (s != ARIA_OK) return s;
+  const size_t need = fused_ws_bytes(M, K);
+  if (need > kNoAllocScratchBytes)
+    return fail(ARIA_ERR_UNSUPPORTED,
+                "M=%lld K=%lld needs %zu bytes of scratch; the static scratch holds %zu "
+                "(256 + 4*M rounded up to 256 + M*K must fit)",
+                (long long)M, (long long)K, need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != ARIA_OK) return s;
+  // the grid barrier's words must start at zero; the array keeps whatever
+  // the last call left (a call that gave up leaves them non-zero)
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch's barrier");
+  const FusedWs ws = fused_ws(scratch, M);
+  return qgemm_impl(aria::kW8A8, M, N, K, ws.xq, ws.sx, Wq, sw, bias, steer_vec, alpha, alpha_dev, Y,
+                    static_cast<cudaStream_t>(stream), X, &ws);
+}
+
 ARIA_API aria_status aria_qgemm_s32(int64_t M, int64_t N, int64_t K, const int8_t* Xq,
                                     const int8_t* Wq, int32_t* C, void* stream) {
   if (!Xq || !Wq || !C) return fail(ARIA_ERR_INVALID_ARG, "NULL device pointer");

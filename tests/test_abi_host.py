@@ -332,3 +332,13 @@ def test_selftest_rules(lib):
     assert f(4, 16, 16, OK_PTR, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 4000001, None) == 1    # above 4 s
     assert f(4, 16, 16, OK_PTR, OK_PTR, ctypes.c_void_p(0x10008), OK_PTR, OK_PTR, 1000, None) == 3
     assert f(4, 24, 16, OK_PTR, OK_PTR, OK_PTR, OK_PTR, OK_PTR, 1000, None) == 2       # N % 16
+
+
+def test_noalloc_refuses_sizes_beyond_its_scratch_before_any_launch(lib):
+    """The static scratch holds 32 MiB: a call whose codes would not fit is
+    refused on the host (no CUDA call is made), with the limit in the message."""
+    f = lib.aria_qgemm_w8a8_fused_noalloc
+    assert f(4096, 16, 16384, OK_PTR, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, None) == 2
+    assert b"scratch" in lib.aria_last_error_message()
+    assert f(4, 16, 16, None, OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, None) == 1
+    assert f(4, 16, 16, ctypes.c_void_p(0x10008), OK_PTR, OK_PTR, None, None, 0.0, None, OK_PTR, None) == 3
