@@ -894,7 +894,7 @@ ARIA_API int aria_trace_read(void* host, size_t bytes) {
   return static_cast<int>(cudaMemcpyFromSymbol(host, aria::g_trace, bytes));
 }
 ARIA_API int aria_trace_clear(void) {
-  static long long zero[8192 * 16];
+  static long long zero[8192 * 24];
   return static_cast<int>(cudaMemcpyToSymbol(aria::g_trace, zero, sizeof(zero)));
 }
 #endif

@@ -22,7 +22,7 @@ constexpr unsigned kStatusTimeout = 1u;
 // stamps of pipeline milestones, read back with aria_trace_read(). Compiled
 // out otherwise.
 #ifdef ARIA_TRACE
-__device__ long long g_trace[8192][16];
+__device__ long long g_trace[8192][24];
 #define ARIA_STAMP(slot)                                                                   \
   do {                                                                                     \
     const int cta_ = ((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) & 8191; \

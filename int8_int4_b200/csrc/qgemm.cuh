@@ -492,36 +492,60 @@ __device__ __noinline__ bool grid_barrier(unsigned* gbar, unsigned ctas, volatil
       *abort = 1;
       return false;
     }
-    __nanosleep(64);
   }
   return true;
 }
 
+// `wmax`: kThreads/32 floats of shared memory not in use at this point
 template <int KIND>
-__device__ __forceinline__ void fused_act_quant(const GemmParams& p, volatile int* abort) {
+__device__ __forceinline__ void fused_act_quant(const GemmParams& p, volatile int* abort,
+                                                float* wmax) {
   constexpr int kWarps = KindTraits<KIND>::kThreads / 32;
   const unsigned ctas = gridDim.x * gridDim.y;
   const unsigned b = blockIdx.y * gridDim.x + blockIdx.x;
   const int rb0 = static_cast<int>(static_cast<int64_t>(p.M) * b / ctas);
   const int rb1 = static_cast<int>(static_cast<int64_t>(p.M) * (b + 1) / ctas);
+  const int rows = rb1 - rb0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = p.K >> 3;  // 16-byte chunks per row
-  for (int r = rb0 + warp; r < rb1; r += kWarps) {
-    const uint4* xr = reinterpret_cast<const uint4*>(p.xf16 + static_cast<int64_t>(r) * p.K);
+  // a CTA's few rows are spread over all its warps: wpr warps per row
+  const int wpr = rows >= 12 ? 1 : rows >= 6 ? 2 : rows >= 3 ? 4 : rows == 2 ? 6 : 12;
+  const int slots = kWarps / wpr;                   // rows quantised side by side
+  const int slot = warp / wpr;
+  const int tr = (warp % wpr) * 32 + lane, tpr = wpr * 32;
+  for (int r0 = rb0; r0 < rb1; r0 += slots) {       // the same rounds in every warp
+    const int r = r0 + slot;
+    const bool live = slot < slots && r < rb1;
+    const uint4* xr = reinterpret_cast<const uint4*>(p.xf16 + static_cast<int64_t>(live ? r : rb0) * p.K);
     float a = 0.0f;
-    for (int c = lane; c < nch; c += 32) a = fmaxf(a, absmax8(__ldg(xr + c)));
+    if (live)
+      for (int c = tr; c < nch; c += tpr) a = fmaxf(a, absmax8(__ldg(xr + c)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const float s = __fdiv_rn(a, 127.0f);
-    uint2* qr = reinterpret_cast<uint2*>(p.xq_ws + static_cast<int64_t>(r) * p.K);
-    for (int c = lane; c < nch; c += 32) qr[c] = quant8_i8(__ldg(xr + c), s, a == 0.0f);
-    if (lane == 0) p.sx_ws[r] = s;
+    if (lane == 0) wmax[warp] = a;
+    __syncthreads();
+    if (live) {
+      for (int w = slot * wpr; w < slot * wpr + wpr; ++w) a = fmaxf(a, wmax[w]);
+      const float s = __fdiv_rn(a, 127.0f);
+      uint2* qr = reinterpret_cast<uint2*>(p.xq_ws + static_cast<int64_t>(r) * p.K);
+      for (int c = tr; c < nch; c += tpr) qr[c] = quant8_i8(__ldg(xr + c), s, a == 0.0f);
+      if (tr == 0) p.sx_ws[r] = s;
+    }
+    __syncthreads();                                // wmax is reused by the next round
   }
-  // the codes are read by other CTAs' TMA loads (async proxy)
-  __threadfence();
+  if (threadIdx.x == 0) ARIA_STAMP(13);
+  // The codes are read by other CTAs' TMA loads (async proxy): each thread
+  // orders its stores toward the async proxy, the CTA meets, and one thread
+  // makes them visible at GPU scope (the fence is cumulative over the
+  // barrier) and arrives at the grid barrier.
   asm volatile("fence.proxy.async.global;" ::: "memory");
   __syncthreads();
-  if (threadIdx.x == 0) grid_barrier(p.gbar, ctas, abort);
+  if (threadIdx.x == 0) {
+    ARIA_STAMP(14);
+    __threadfence();
+    grid_barrier(p.gbar, ctas, abort);
+    ARIA_STAMP(15);
+  }
   __syncthreads();
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -591,7 +615,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     mbar_init(mma_drain, 1);
     mbar_init(acc_last, 1);
     *abort_flag = 0;
+    ARIA_STAMP(16);
     fence_mbar_init();
+    ARIA_STAMP(17);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
@@ -601,10 +627,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
+    if (lane == 0) ARIA_STAMP(18);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) ARIA_STAMP(19);
   const uint32_t tmem_base = *tmem_slot;
   // Programmatic dependent launch: this CTA may start while the preceding
   // kernel in the stream drains. Packed weights and their scales are inputs
@@ -658,7 +686,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
   if constexpr (KIND == kW8A8) {
-    if (p.xf16) fused_act_quant<KIND>(p, abort_flag);
+    if (p.xf16) fused_act_quant<KIND>(p, abort_flag, reinterpret_cast<float*>(smem + p.off_sxd));
   }
   if (threadIdx.x == 0) ARIA_STAMP(2);
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
@@ -1023,17 +1051,27 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           }
         }
         if constexpr (KIND == kW8A8) {
-          // rare elements: re-sum the partials and round exactly; these later
-          // stores of the same thread replace the values written above
+          // rare elements: round exactly from the summed accumulator (picked
+          // from registers by index: no second trip to the peers' shared
+          // memory); these later stores of the same thread replace the
+          // values written above
           while (rare_mask) {
             const int idx = __ffs(rare_mask) - 1;
             rare_mask &= rare_mask - 1;
             const int u = idx >> 2, k = idx & 3;
             const int ml = ml0 + u * kWarps;
             const int m = m0 + ml;
-            int32_t a = 0;
-            for (int q = 0; q < p.splits; ++q)
-              a += static_cast<int32_t>(ld_dsmem_u32(mapa_shared(red_u32 + static_cast<uint32_t>((ml * 128 + nl + k) * 4), q)));
+            uint32_t asel = 0u;
+#pragma unroll
+            for (int uu = 0; uu < kRows; ++uu) {
+              if (uu == u) {
+                const uint32_t c4[4] = {acc[uu].x, acc[uu].y, acc[uu].z, acc[uu].w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  if (kk == k) asel = c4[kk];
+              }
+            }
+            const int32_t a = static_cast<int32_t>(asel);
             const RowConst<kW8A8> rk = row_const<kW8A8>(n + k, p);
             reinterpret_cast<__half*>(p.Y)[static_cast<int64_t>(m) * p.N + n + k] =
                 epi_w8a8(a, __ldg(p.sx + m), rk);
