@@ -164,6 +164,30 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
     if (best_mt == 0) best_mt = K <= 2048 ? mt0 + 1 : mt0;
     mt = tile_for(best_mt, &bn);
   }
+  // Many tokens (several tiles per CTA): the persistent CTAs take the tiles
+  // round-robin, so the slowest CTA does ceil(tiles / SMs) of them. Pick the
+  // token tile (a multiple of 16 in [128, 256]) that minimises that count
+  // times the tile's width plus a fixed per-tile cost (16 token-columns'
+  // worth), e.g. 176 instead of 256 for N = 1536 at M = 4096: 288 tiles in
+  // two nearly full waves instead of 192 in two waves of which one is 30 %
+  // full.
+  bool wave_policy = M > 512;
+#if defined(ARIA_MAX_BN)
+  wave_policy = false;  // tuning builds pin the tile
+#endif
+  if (wave_policy) {
+    int64_t best_cost = -1;
+    for (int b = 256; b >= 128; b -= 16) {
+      const int64_t m_t = (M + b - 1) / b;
+      const int64_t waves = (static_cast<int64_t>(nt) * m_t + di.sms - 1) / di.sms;
+      const int64_t cost = waves * (b + 16);
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        bn = b;
+        mt = static_cast<int>(m_t);
+      }
+    }
+  }
   p.BN = bn;
   const int64_t tiles = static_cast<int64_t>(nt) * mt;
   if (tiles > (int64_t{1} << 30)) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
@@ -180,6 +204,12 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.splits = splits;
 
   const bool dq = (kind == kQ8 || kind == kQ4);
+  // q8/q4 with one tile per CTA (every split-K CTA has one too): the A
+  // operand lives in tensor memory, so a stage holds only the activation
+  // tile; the ring depth stays <= 8 (8 A slots of 32 TMEM columns)
+  const bool ta = dq && tiles <= di.sms;
+  p.tmem_a = ta ? 1 : 0;
+  const uint32_t a_tile = ta ? 0u : kATile;
   const uint32_t out_bytes = kind == kS32 ? 4 : 2;
   const uint32_t epi_warps = dq ? 4 : 8;
   const uint32_t stage_bytes = epi_warps * 2 * kEpiRows * 32 * out_bytes;  // 2 store boxes per warp
@@ -191,7 +221,7 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   // stage ring: one A tile + one X tile per stage (one MMA commit each);
   // q8/q4 also keep a ring of raw packed weight tiles for the dequant warps
   int nr = 0, na = 0, nx = 0;
-  const int64_t st_bytes = kATile + p.x_stage;
+  const int64_t st_bytes = a_tile + p.x_stage;
   for (int k = 8; k >= 2 && na == 0; --k) {
     if (!dq) {
       if (k * st_bytes <= budget) na = k;
@@ -211,7 +241,7 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.n_x = nx;
   p.off_raw = 0;
   p.off_a = p.off_raw + nr * p.raw_stage;
-  p.off_x = p.off_a + na * kATile;
+  p.off_x = p.off_a + na * a_tile;
   p.off_stage = p.off_x + nx * p.x_stage;
   p.off_sxd = p.off_stage + stage_bytes;
   p.off_bar = p.off_sxd + sxd_bytes;

@@ -28,7 +28,11 @@
 //                accumulator buffer (W8A8 and fp16 use warps 8..11 for it as well)
 //   warps 8..11  q8/q4: dequantise raw weights into fp16 A tiles (one weight
 //                row per thread; exact int8 -> fp16; fp16 code*scale for q4);
-//                they take part in the epilogue of the CTA's last tile
+//                they take part in the epilogue of the CTA's last tile. When
+//                each CTA has one tile, the A tiles are written to tensor
+//                memory (tcgen05.st, a row per TMEM lane) and the MMA reads A
+//                from there: shared memory then holds only the activation and
+//                raw-weight rings, which can be nearly twice as deep
 // Rings of shared-memory stages with mbarriers connect the roles; every wait
 // is bounded. Split-K (few output tiles): a cluster of S CTAs shares one tile,
 // each taking a contiguous K range; all warps then sum the partial
@@ -81,6 +85,10 @@ struct GemmParams {
   // first stage of each CTA's first tile so that the waits on it run out
   uint64_t wait_ns;
   int drop_first_stage;
+  // q8/q4 with one tile per CTA: the dequantised weights (the MMA's A
+  // operand) go to tensor memory, columns [kAccCols + 32 s, +32) for stage s,
+  // instead of shared memory; the accumulator keeps columns [0, BN)
+  int tmem_a;
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
@@ -790,14 +798,21 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         if (!(ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4, wlim))) break;
         if (kb == 0 && ti == 0 && lane == 0) ARIA_STAMP(4);
         tc_fence_after();
-        const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
         const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sa * p.x_stage));
+        if (T::kDequant && p.tmem_a) {
+          // A: this stage's 32 TMEM columns (8 per 16-wide K step)
+          const uint32_t at = tmem_base + kAccCols + static_cast<uint32_t>(sa) * 32u;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
-          if constexpr (T::kMmaF16)
-            umma_f16_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
-          else
-            umma_i8_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+          for (int j = 0; j < 4; ++j) umma_f16_ts_elect(dt, at + 8 * j, bd + 2 * j, idesc, (kb | j) != 0);
+        } else {
+          const uint64_t ad = sdesc_sw128(smem_u32(abuf + sa * kATile));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {  // 4 x 32 bytes of K per 128-byte block
+            if constexpr (T::kMmaF16)
+              umma_f16_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+            else
+              umma_i8_elect(dt, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+          }
         }
         umma_commit_elect(st_empty + sa);  // releases both tiles of the stage
         if (++sa == p.n_a) { sa = 0; ph ^= 1u; }
@@ -834,6 +849,45 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
 #pragma unroll
           for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
             if (!(ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7, wlim))) break;
+            if (p.tmem_a) {
+              // the MMA that read this slot has completed (its commit arrived)
+              tc_fence_after();
+              uint32_t o[32];  // TMEM column c = fp16 pair (k = 2c, 2c + 1) of this K block
+              if constexpr (KIND == kQ8) {
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                  const uint4 w = v[4 * h + cc];
+                  i8x4_to_h(w.x, o[8 * cc + 0], o[8 * cc + 1]);
+                  i8x4_to_h(w.y, o[8 * cc + 2], o[8 * cc + 3]);
+                  i8x4_to_h(w.z, o[8 * cc + 4], o[8 * cc + 5]);
+                  i8x4_to_h(w.w, o[8 * cc + 6], o[8 * cc + 7]);
+                }
+              } else {
+                const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                  const int c = 2 * h + g;
+                  const uint32_t spair = scw[c >> 1];
+                  const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
+                  const uint4 w = v[c];
+                  const uint4 q0 = nib8_to_h(w.x, s2), q1 = nib8_to_h(w.y, s2);
+                  const uint4 q2 = nib8_to_h(w.z, s2), q3 = nib8_to_h(w.w, s2);
+                  o[16 * g + 0] = q0.x; o[16 * g + 1] = q0.y; o[16 * g + 2] = q0.z; o[16 * g + 3] = q0.w;
+                  o[16 * g + 4] = q1.x; o[16 * g + 5] = q1.y; o[16 * g + 6] = q1.z; o[16 * g + 7] = q1.w;
+                  o[16 * g + 8] = q2.x; o[16 * g + 9] = q2.y; o[16 * g + 10] = q2.z; o[16 * g + 11] = q2.w;
+                  o[16 * g + 12] = q3.x; o[16 * g + 13] = q3.y; o[16 * g + 14] = q3.z; o[16 * g + 15] = q3.w;
+                }
+              }
+              __syncwarp();  // tcgen05.st is warp-collective
+              tmem_st32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCols +
+                            static_cast<uint32_t>(sa) * 32u,
+                        o);
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(st_full + sa);
+              if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
+              continue;
+            }
             uint8_t* dst = abuf + sa * kATile;
             if constexpr (KIND == kQ8) {
               // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
