@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -188,6 +189,27 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
       }
     }
   }
+  // W8A8 with few weight-row tiles and a short K: the narrowest token tile
+  // that still leaves at least two thirds of the SMs busy without split-K
+  // (measured at M = 432, N = K = 1536: 48-token tiles 6.8 us against 9.3 us
+  // for 144-token tiles in 3-way split-K clusters; at K = 6144 the split
+  // stays faster)
+  bool narrow_policy = kind == kW8A8 && M <= 512 && K <= 2048 && static_cast<int64_t>(nt) * mt < di.sms;
+#if defined(ARIA_MAX_BN)
+  narrow_policy = false;  // tuning builds pin the tile
+#endif
+  if (narrow_policy) {
+    for (int b = bn - 16; b >= 48; b -= 16) {
+      const int64_t m_t = (M + b - 1) / b;
+      const int64_t t = static_cast<int64_t>(nt) * m_t;
+      if (t > di.sms) break;
+      if (3 * t >= 2 * static_cast<int64_t>(di.sms)) {
+        bn = b;
+        mt = static_cast<int>(m_t);
+        break;
+      }
+    }
+  }
   p.BN = bn;
   const int64_t tiles = static_cast<int64_t>(nt) * mt;
   if (tiles > (int64_t{1} << 30)) return fail(ARIA_ERR_UNSUPPORTED, "too many tiles");
@@ -213,7 +235,7 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   const uint32_t out_bytes = kind == kS32 ? 4 : 2;
   const uint32_t epi_warps = dq ? 4 : 8;
   const uint32_t stage_bytes = epi_warps * 2 * kEpiRows * 32 * out_bytes;  // 2 store boxes per warp
-  const uint32_t sxd_bytes = 256 * 4;
+  const uint32_t sxd_bytes = 2 * aria::kTileBnMax * 4;  // W8A8 token scales, two m-tiles
   p.x_stage = static_cast<uint32_t>(bn) * 128u;
   p.raw_stage = kind == kQ8 ? kATile : (kind == kQ4 ? kATile + kQ4ScaleTile : 0);
   p.raw_stage = (p.raw_stage + 1023u) & ~1023u;
@@ -222,7 +244,11 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   // q8/q4 also keep a ring of raw packed weight tiles for the dequant warps
   int nr = 0, na = 0, nx = 0;
   const int64_t st_bytes = a_tile + p.x_stage;
-  for (int k = 8; k >= 2 && na == 0; --k) {
+  int k_max = 8;
+#if defined(ARIA_MAX_STAGES)
+  k_max = ARIA_MAX_STAGES;  // tuning builds only
+#endif
+  for (int k = k_max; k >= 2 && na == 0; --k) {
     if (!dq) {
       if (k * st_bytes <= budget) na = k;
       continue;
@@ -257,6 +283,15 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   out->smem = smem;
   return ARIA_OK;
 }
+
+// Trace builds: each GEMM launch gets the next trace row block (see
+// ARIA_STAMP); 0 otherwise.
+#ifdef ARIA_TRACE
+std::atomic<int> g_trace_launches{0};
+int next_trace_launch() { return g_trace_launches.fetch_add(1); }
+#else
+int next_trace_launch() { return 0; }
+#endif
 
 // programmatic dependent launch: the kernel may start while the previous
 // kernel in the stream drains; it waits (griddepcontrol.wait) before reading
@@ -351,6 +386,7 @@ aria_status launch_gemm(const Plan& pl, const CUtensorMap& tw, const CUtensorMap
     cfg.attrs = attr;
   }
   set_pdl(cfg, attr);
+  prm.trace_launch = next_trace_launch();
   cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tw, ts, tx, prm);
   if (e != cudaSuccess) return cuda_fail(e, "qgemm launch");
   return ARIA_OK;
@@ -429,7 +465,8 @@ bool small_layout(int kind, int64_t M, int64_t N, int64_t K, int S, int clusters
   p->off_part = static_cast<uint32_t>(up(off, 128));
   off = p->off_part + (S > 1 ? static_cast<uint64_t>(tb) * 8 * (p->r_pad + 4) * 4 : 0);
   p->off_bar = static_cast<uint32_t>(up(off, 16));
-  *smem = p->off_bar + 16;
+  p->off_sw = p->off_bar + 16;  // q8 channel scales of the rows
+  *smem = p->off_sw + static_cast<uint64_t>(rmax) * 4;
   (void)M;
   return *smem <= kSmallSmemBudget;
 }
@@ -508,7 +545,9 @@ aria_status launch_small_t(const SmallPlan& pl, cudaStream_t st) {
     cfg.attrs = attr;
   }
   set_pdl(cfg, attr);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, pl.p);
+  aria::SmallParams sp = pl.p;
+  sp.trace_launch = next_trace_launch();
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, sp);
   if (e != cudaSuccess) return cuda_fail(e, "few-token GEMM launch");
   return ARIA_OK;
 }
@@ -925,6 +964,7 @@ ARIA_API int aria_trace_read(void* host, size_t bytes) {
 }
 ARIA_API int aria_trace_clear(void) {
   static long long zero[8192 * 24];
+  g_trace_launches = 0;
   return static_cast<int>(cudaMemcpyToSymbol(aria::g_trace, zero, sizeof(zero)));
 }
 #endif

@@ -19,20 +19,32 @@ __device__ unsigned int g_wait_site;
 constexpr unsigned kStatusTimeout = 1u;
 
 // Optional phase tracing (compile with -DARIA_TRACE): per-CTA %globaltimer
-// stamps of pipeline milestones, read back with aria_trace_read(). Compiled
-// out otherwise.
+// stamps of pipeline milestones, read back with aria_trace_read(). Rows
+// [2048 j, 2048 j + 2048) hold launch j (mod 4) since the last
+// aria_trace_clear(), so a chain of launches can be followed; the kernel
+// parameters `p` carry j. Compiled out otherwise.
 #ifdef ARIA_TRACE
 __device__ long long g_trace[8192][24];
 #define ARIA_STAMP(slot)                                                                   \
   do {                                                                                     \
-    const int cta_ = ((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) & 8191; \
+    const int cta_ = (((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) & 2047) + \
+                     2048 * (p.trace_launch & 3);                                          \
     long long t_;                                                                          \
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                 \
     g_trace[cta_][(slot)] = t_;                                                            \
   } while (0)
+#define ARIA_TRACE_VAL(slot, v)                                                            \
+  do {                                                                                     \
+    const int cta_ = (((blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x) & 2047) + \
+                     2048 * (p.trace_launch & 3);                                          \
+    g_trace[cta_][(slot)] = static_cast<long long>(v);                                     \
+  } while (0)
 #else
 #define ARIA_STAMP(slot) \
   do {                   \
+  } while (0)
+#define ARIA_TRACE_VAL(slot, v) \
+  do {                          \
   } while (0)
 #endif
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
@@ -42,6 +54,20 @@ __device__ __forceinline__ uint64_t globaltimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+// Trace builds: total time a role spends in one kind of wait (written with
+// ARIA_TRACE_VAL); nothing otherwise.
+struct WaitClock {
+#ifdef ARIA_TRACE
+  uint64_t total = 0, t0 = 0;
+  __device__ __forceinline__ void start() { t0 = globaltimer(); }
+  __device__ __forceinline__ void stop() { total += globaltimer() - t0; }
+#else
+  uint64_t total = 0;
+  __device__ __forceinline__ void start() {}
+  __device__ __forceinline__ void stop() {}
+#endif
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -346,6 +372,27 @@ __device__ __forceinline__ void pdl_wait() {
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// Loads of data that the preceding kernel in the stream may have written
+// (activations, token scales, steering vectors, unpacked weights). They stay
+// after the dependency wait (griddepcontrol.wait below): volatile inline
+// asm keeps its program order with that wait, whereas the compiler treats
+// read-only-cache loads (__ldg) as loads of invariant memory and may hoist
+// them above it.
+__device__ __forceinline__ uint4 ld_dep_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float ld_dep_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 
 // 2-D tiled prefetch into L2 (no shared memory, no completion tracking)
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int32_t c0, int32_t c1) {

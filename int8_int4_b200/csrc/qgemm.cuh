@@ -32,7 +32,10 @@
 //                each CTA has one tile, the A tiles are written to tensor
 //                memory (tcgen05.st, a row per TMEM lane) and the MMA reads A
 //                from there: shared memory then holds only the activation and
-//                raw-weight rings, which can be nearly twice as deep
+//                raw-weight rings, which can be nearly twice as deep; for
+//                q4, warps 4..7, idle until the tile's accumulator is
+//                complete, dequantise the odd K blocks while warps 8..11
+//                take the even ones
 // Rings of shared-memory stages with mbarriers connect the roles; every wait
 // is bounded. Split-K (few output tiles): a cluster of S CTAs shares one tile,
 // each taking a contiguous K range; all warps then sum the partial
@@ -55,6 +58,7 @@ constexpr uint32_t kATile = 16384;       // 128 rows x 128 bytes
 constexpr uint32_t kQ4ScaleTile = 2048;  // 128 rows x 8 fp16 scales
 constexpr uint32_t kAccCols = 256;       // TMEM columns per accumulator buffer
 constexpr int kEpiRows = 16;             // tokens per epilogue store box
+constexpr int kTileBnMax = 256;          // largest token tile (MMA N)
 constexpr int kL2Ahead = 4;              // weight units prefetched into L2 ahead of the TMA loads
 
 struct GemmParams {
@@ -89,6 +93,7 @@ struct GemmParams {
   // operand) go to tensor memory, columns [kAccCols + 32 s, +32) for stage s,
   // instead of shared memory; the accumulator keeps columns [0, BN)
   int tmem_a;
+  int trace_launch;       // trace builds: the launch's index since the trace was cleared
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
 
@@ -166,33 +171,57 @@ __device__ __forceinline__ float steer_alpha(const GemmParams& p) {
   return p.alpha_dev ? *p.alpha_dev : p.alpha;
 }
 
+// The per-channel inputs of the epilogue as loaded (no arithmetic on them
+// yet), so that a CTA can issue the loads for its next tile early and use
+// them a tile later.
+struct RowRaw {
+  float sw = 0.0f, v = 0.0f;
+  unsigned short bias = 0;  // fp16 bits
+};
+
 template <int KIND>
-__device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) {
+__device__ __forceinline__ RowRaw row_raw(int n, const GemmParams& p) {
+  RowRaw r;
+  if (n >= p.N) return r;
+  if constexpr (KIND == kW8A8 || KIND == kQ8) r.sw = __ldg(p.sw + n);
+  if (p.bias) r.bias = __half_as_ushort(p.bias[n]);
+  if (p.steer) r.v = ld_dep_f32(p.steer + n);
+  return r;
+}
+
+// `alpha`: the launch's steering strength (steer_alpha), 0 without steering
+template <int KIND>
+__device__ __forceinline__ RowConst<KIND> row_const_from(const RowRaw& r, int n, const GemmParams& p,
+                                                        float alpha) {
   RowConst<KIND> c;
   if (n >= p.N) return c;
   c.has_bias = p.bias != nullptr;
-  const float alpha = p.steer ? steer_alpha(p) : 0.0f;
   c.has_steer = p.steer != nullptr && alpha != 0.0f;
   if constexpr (KIND == kW8A8) {
-    c.sw = __ldg(p.sw + n);
+    c.sw = r.sw;
     c.sw_up = __fmul_rn(c.sw, 1.0f + 0x1p-21f);
     c.sw_dn = __fmul_rn(c.sw, 1.0f - 0x1p-21f);
-    if (c.has_bias) c.bias = __half2float(p.bias[n]);
+    if (c.has_bias) c.bias = __half2float(__ushort_as_half(r.bias));
     if (c.has_steer) {
       c.alpha = alpha;
-      c.v = __ldg(p.steer + n);
+      c.v = r.v;
       c.av_hi = __fmul_rn(c.alpha, c.v);
       c.av_lo = __fmaf_rn(c.alpha, c.v, -c.av_hi);  // exact remainder of the product
     }
   } else {
-    if constexpr (KIND == kQ8) c.sw = __ldg(p.sw + n);
-    if (c.has_bias) c.bias = __half2float(p.bias[n]);
+    if constexpr (KIND == kQ8) c.sw = r.sw;
+    if (c.has_bias) c.bias = __half2float(__ushort_as_half(r.bias));
     if (c.has_steer) {
       c.alpha = alpha;
-      c.v = __ldg(p.steer + n);
+      c.v = r.v;
     }
   }
   return c;
+}
+
+template <int KIND>
+__device__ __forceinline__ RowConst<KIND> row_const(int n, const GemmParams& p) {
+  return row_const_from<KIND>(row_raw<KIND>(n, p), n, p, p.steer ? steer_alpha(p) : 0.0f);
 }
 
 // W8A8 reference sequence: ((acc * s_x) * s_w) + bias + alpha*v in fp64, each
@@ -458,6 +487,33 @@ __device__ __forceinline__ void epilogue_chunk_store(int c, int nb, int m0, int 
     }
 }
 
+// The calling warp's chunks c_first, c_first + cs, ... < nchunk of one
+// accumulator buffer (`tacc`: its 32 TMEM lanes). After the last TMEM read,
+// `release()` runs (warp-uniform; the buffer may then be reused). Store boxes
+// alternate between the two halves of `sb0`, `nst` counting the boxes used
+// so far. Returns the new count. (Loading the next chunk from TMEM while the
+// current one is converted measured slower: 36.6 against 33.8 us at
+// M = 4096, N = 4608, K = 1536.)
+template <int KIND, class Release>
+__device__ __forceinline__ int epilogue_chunks(int c_first, int cs, int nchunk, uint32_t tacc, int lane,
+                                               uint8_t* sb0, int nst, const RowConst<KIND>& rc,
+                                               const float* sxs, int nb, int m0, const GemmParams& p,
+                                               Release release) {
+  using T = KindTraits<KIND>;
+  if (c_first >= nchunk) {
+    release();
+    return nst;
+  }
+  for (int c = c_first; c < nchunk; c += cs) {
+    uint8_t* sbuf = sb0 + (nst & 1) * T::kStageBuf;
+    epilogue_chunk_compute<KIND>(c, tacc, lane, sbuf, rc, sxs);
+    if (c + cs >= nchunk) release();
+    epilogue_chunk_store<KIND>(c, nb, m0, lane, sbuf, p);
+    ++nst;
+  }
+  return nst;
+}
+
 // ----------------------------------------------- fused activation quant ---
 // "Results" (aria project page): W8A8 quantises the activations per token to
 // 8 bits. In the fused form every CTA of the GEMM quantises a share of the
@@ -494,6 +550,7 @@ __device__ __noinline__ bool grid_barrier(unsigned* gbar, unsigned ctas, volatil
   }
   const uint64_t t0 = globaltimer();
   while (ld_acquire_gpu(gen) == g0) {
+    __nanosleep(64);  // fewer polls of the line the arrivals update
     if (globaltimer() - t0 > kWaitLimitNs) {
       atomicOr(&g_status, kStatusTimeout);
       atomicExch(&g_wait_site, 30u);
@@ -527,7 +584,7 @@ __device__ __forceinline__ void fused_act_quant(const GemmParams& p, volatile in
     const uint4* xr = reinterpret_cast<const uint4*>(p.xf16 + static_cast<int64_t>(live ? r : rb0) * p.K);
     float a = 0.0f;
     if (live)
-      for (int c = tr; c < nch; c += tpr) a = fmaxf(a, absmax8(__ldg(xr + c)));
+      for (int c = tr; c < nch; c += tpr) a = fmaxf(a, absmax8(ld_dep_v4(xr + c)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     if (lane == 0) wmax[warp] = a;
@@ -536,7 +593,7 @@ __device__ __forceinline__ void fused_act_quant(const GemmParams& p, volatile in
       for (int w = slot * wpr; w < slot * wpr + wpr; ++w) a = fmaxf(a, wmax[w]);
       const float s = __fdiv_rn(a, 127.0f);
       uint2* qr = reinterpret_cast<uint2*>(p.xq_ws + static_cast<int64_t>(r) * p.K);
-      for (int c = tr; c < nch; c += tpr) qr[c] = quant8_i8(__ldg(xr + c), s, a == 0.0f);
+      for (int c = tr; c < nch; c += tpr) qr[c] = quant8_i8(ld_dep_v4(xr + c), s, a == 0.0f);
       if (tr == 0) p.sx_ws[r] = s;
     }
     __syncthreads();                                // wmax is reused by the next round
@@ -587,7 +644,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   uint8_t* abuf = smem + p.off_a;
   uint8_t* xbuf = smem + p.off_x;
   uint8_t* stage = smem + p.off_stage;
-  float* sxs = reinterpret_cast<float*>(smem + p.off_sxd);   // s_x of the current m-tile
+  float* sxs = reinterpret_cast<float*>(smem + p.off_sxd);   // s_x of two m-tiles [2][kTileBnMax]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   // one stage = an A tile (weights, 128 rows x 128 B of K) and an X tile
   // (activations, BN rows x 128 B of K); one commit releases both
@@ -609,7 +666,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.n_raw; ++i) {
       mbar_init(raw_full + i, 1);
-      mbar_init(raw_empty + i, 128);
+      mbar_init(raw_empty + i, (KIND == kQ4 && p.tmem_a) ? 256 : 128);  // the dequant threads
     }
     for (int i = 0; i < p.n_a; ++i) {
       // q8/q4: 128 dequant threads + the X producer; W8A8: the single producer
@@ -625,7 +682,6 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     *abort_flag = 0;
     ARIA_STAMP(16);
     fence_mbar_init();
-    ARIA_STAMP(17);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmW);
@@ -699,6 +755,131 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   if (threadIdx.x == 0) ARIA_STAMP(2);
   bool epi_ok = true;               // split-K: this CTA's accumulator is complete
 
+  // Dequantisation of the raw weight ring into A stages by 128 threads, one
+  // weight row each (t = row within the tile). `ngrp` groups of 128
+  // threads share the work: group `grp` takes the K blocks kb with
+  // kb % ngrp == grp (every raw stage holds an even number of K blocks).
+  auto dequant_rows = [&](const int t, const int grp, const int ngrp) -> bool {
+    int s = 0, sa = 0;  // raw ring slot, stage ring slot
+    uint32_t rph = 0, aph = 0;
+    bool ok = true;
+    WaitClock wc_raw, wc_empty;  // trace builds: time waiting for weights / for a free stage
+    for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
+      for (int i = 0; i < nu && ok; ++i) {
+        wc_raw.start();
+        ok = mbar_wait_fast(raw_full + s, rph, abort_flag, 6, wlim);
+        wc_raw.stop();
+        if (!ok) break;
+        if (t == 0 && grp == 0 && tile == tile0 && i == 0) ARIA_STAMP(12);
+        const uint8_t* src = raw + s * p.raw_stage;
+        uint4 v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // the 16-byte chunks of this group's K blocks
+          v[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (ngrp == 1 || (c / (8 / T::kKbPerUnit)) % 2 == grp)
+            v[c] = *reinterpret_cast<const uint4*>(src + sw128(t, c));
+        }
+        uint4 sc = make_uint4(0, 0, 0, 0);
+        if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
+        // The slot's next writer is a TMA load (async proxy): order this
+        // thread's generic-proxy reads of it before that write. Without
+        // the proxy fence the release of the arrive alone let a refill land
+        // before the reads of v[4..7] completed (measured: wrong second A
+        // tile of a unit in about 1 of 3 launches at M = 4096).
+        fence_proxy_async_smem();
+        mbar_arrive(raw_empty + s);
+        if (++s == p.n_raw) { s = 0; rph ^= 1u; }
+#pragma unroll
+        for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
+          if (ngrp == 2 && h % 2 != grp) {  // the other group's K block
+            if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
+            continue;
+          }
+          wc_empty.start();
+          ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7, wlim);
+          wc_empty.stop();
+          if (!ok) break;
+          if (p.tmem_a) {
+            // the MMA that read this slot has completed (its commit arrived)
+            tc_fence_after();
+            uint32_t o[32];  // TMEM column c = fp16 pair (k = 2c, 2c + 1) of this K block
+            if constexpr (KIND == kQ8) {
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                const uint4 w = v[4 * h + cc];
+                i8x4_to_h(w.x, o[8 * cc + 0], o[8 * cc + 1]);
+                i8x4_to_h(w.y, o[8 * cc + 2], o[8 * cc + 3]);
+                i8x4_to_h(w.z, o[8 * cc + 4], o[8 * cc + 5]);
+                i8x4_to_h(w.w, o[8 * cc + 6], o[8 * cc + 7]);
+              }
+            } else {
+              const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
+#pragma unroll
+              for (int g = 0; g < 2; ++g) {
+                const int c = 2 * h + g;
+                const uint32_t spair = scw[c >> 1];
+                const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
+                const uint4 w = v[c];
+                const uint4 q0 = nib8_to_h(w.x, s2), q1 = nib8_to_h(w.y, s2);
+                const uint4 q2 = nib8_to_h(w.z, s2), q3 = nib8_to_h(w.w, s2);
+                o[16 * g + 0] = q0.x; o[16 * g + 1] = q0.y; o[16 * g + 2] = q0.z; o[16 * g + 3] = q0.w;
+                o[16 * g + 4] = q1.x; o[16 * g + 5] = q1.y; o[16 * g + 6] = q1.z; o[16 * g + 7] = q1.w;
+                o[16 * g + 8] = q2.x; o[16 * g + 9] = q2.y; o[16 * g + 10] = q2.z; o[16 * g + 11] = q2.w;
+                o[16 * g + 12] = q3.x; o[16 * g + 13] = q3.y; o[16 * g + 14] = q3.z; o[16 * g + 15] = q3.w;
+              }
+            }
+            __syncwarp();  // tcgen05.st is warp-collective
+            tmem_st32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCols +
+                          static_cast<uint32_t>(sa) * 32u,
+                      o);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(st_full + sa);
+            if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
+            continue;
+          }
+          uint8_t* dst = abuf + sa * kATile;
+          if constexpr (KIND == kQ8) {
+            // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint4 w = v[4 * h + cc];
+              uint4 o0, o1;
+              i8x4_to_h(w.x, o0.x, o0.y);
+              i8x4_to_h(w.y, o0.z, o0.w);
+              i8x4_to_h(w.z, o1.x, o1.y);
+              i8x4_to_h(w.w, o1.z, o1.w);
+              *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc)) = o0;
+              *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc + 1)) = o1;
+            }
+          } else {
+            // raw chunks 2h, 2h+1 (one 32-k group each) -> fp16 chunks 0..7
+            const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int c = 2 * h + g;
+              const uint32_t spair = scw[c >> 1];
+              const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
+              const uint4 w = v[c];
+              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 0)) = nib8_to_h(w.x, s2);
+              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 1)) = nib8_to_h(w.y, s2);
+              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 2)) = nib8_to_h(w.z, s2);
+              *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 3)) = nib8_to_h(w.w, s2);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(st_full + sa);
+          if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
+        }
+      }
+    }
+    if (t == 0 && grp == 0) {
+      ARIA_TRACE_VAL(23, wc_raw.total);
+      ARIA_TRACE_VAL(17, wc_empty.total);
+    }
+    return ok;
+  };
+
   // The producer and MMA roles run as whole converged warps: every lane waits,
   // one lane issues (TMA by lane 0, MMA and commit by elect.sync), so the
   // issue loops stay warp-uniform. Ring slots and phases advance
@@ -707,6 +888,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     // ------------------------------------------------ weight tile producer
     const uint64_t pol = policy_evict_first();  // weights are read once per m-tile
     bool ok = true;
+    WaitClock wc_pe;  // trace builds (W8A8, fp16): time waiting for free stages
     int s = 0;
     uint32_t ph = 0;
     for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
@@ -750,7 +932,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             if (++s == p.n_a) { s = 0; ph ^= 1u; }
             continue;
           }
-          if (!(ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2, wlim))) break;
+          wc_pe.start();
+          ok = mbar_wait_warp(st_empty + s, ph ^ 1, abort_flag, 2, wlim);
+          wc_pe.stop();
+          if (!ok) break;
           if (lane == 0) {
             if (kb + kL2Ahead < nkb) tma_prefetch_2d(&tmW, (u_begin + kb + kL2Ahead) * T::kWUnitX, n0);
             mbar_arrive_expect_tx(st_full + s, kATile + p.x_stage);
@@ -762,6 +947,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           if (++s == p.n_a) { s = 0; ph ^= 1u; }
         }
       }
+    }
+    if constexpr (!T::kDequant) {
+      if (lane == 0) ARIA_TRACE_VAL(17, wc_pe.total);
     }
   } else if (warp == 2 && T::kDequant) {
     // -------------------------------------------- activation tile producer
@@ -788,6 +976,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     int ti = 0, sa = 0;
     uint32_t ph = 0;
     bool ok = true;
+    WaitClock wc_full;  // trace builds: time waiting for full stages
     for (int tile = tile0; tile < p.tiles && ok; tile += tstep, ++ti) {
       const int b = ti & 1;
       if (!(ok = mbar_wait_warp(acc_empty + b, ((ti >> 1) & 1) ^ 1, abort_flag, 9, wlim))) break;
@@ -795,7 +984,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       tc_fence_after();
       const uint32_t dt = tmem_base + b * kAccCols;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!(ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4, wlim))) break;
+        wc_full.start();
+        ok = mbar_wait_warp(st_full + sa, ph, abort_flag, 4, wlim);
+        wc_full.stop();
+        if (!ok) break;
         if (kb == 0 && ti == 0 && lane == 0) ARIA_STAMP(4);
         tc_fence_after();
         const uint64_t bd = sdesc_sw128(smem_u32(xbuf + sa * p.x_stage));
@@ -821,108 +1013,12 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
       if (tile + tstep >= p.tiles) umma_commit_elect(acc_last);
       if (lane == 0) ARIA_STAMP(5);
     }
+    if (lane == 0) ARIA_TRACE_VAL(22, wc_full.total);
   } else if (T::kDequant && warp >= 8) {
     // ------------------------------------------------------ dequantise
     if constexpr (T::kDequant) {
       const int t = threadIdx.x - 256;  // weight row within the tile
-      int s = 0, sa = 0;  // raw ring slot, stage ring slot
-      uint32_t rph = 0, aph = 0;
-      bool ok = true;
-      for (int tile = tile0; tile < p.tiles && ok; tile += tstep) {
-        for (int i = 0; i < nu && ok; ++i) {
-          if (!(ok = mbar_wait_fast(raw_full + s, rph, abort_flag, 6, wlim))) break;
-          if (t == 0 && tile == tile0 && i == 0) ARIA_STAMP(12);
-          const uint8_t* src = raw + s * p.raw_stage;
-          uint4 v[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(src + sw128(t, c));
-          uint4 sc = make_uint4(0, 0, 0, 0);
-          if constexpr (KIND == kQ4) sc = *reinterpret_cast<const uint4*>(src + kATile + t * 16);
-          // The slot's next writer is a TMA load (async proxy): order this
-          // thread's generic-proxy reads of it before that write. Without
-          // the proxy fence the release of the arrive alone let a refill land
-          // before the reads of v[4..7] completed (measured: wrong second A
-          // tile of a unit in about 1 of 3 launches at M = 4096).
-          fence_proxy_async_smem();
-          mbar_arrive(raw_empty + s);
-          if (++s == p.n_raw) { s = 0; rph ^= 1u; }
-#pragma unroll
-          for (int h = 0; h < T::kKbPerUnit; ++h) {  // A tiles produced per raw stage
-            if (!(ok = mbar_wait_fast(st_empty + sa, aph ^ 1, abort_flag, 7, wlim))) break;
-            if (p.tmem_a) {
-              // the MMA that read this slot has completed (its commit arrived)
-              tc_fence_after();
-              uint32_t o[32];  // TMEM column c = fp16 pair (k = 2c, 2c + 1) of this K block
-              if constexpr (KIND == kQ8) {
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                  const uint4 w = v[4 * h + cc];
-                  i8x4_to_h(w.x, o[8 * cc + 0], o[8 * cc + 1]);
-                  i8x4_to_h(w.y, o[8 * cc + 2], o[8 * cc + 3]);
-                  i8x4_to_h(w.z, o[8 * cc + 4], o[8 * cc + 5]);
-                  i8x4_to_h(w.w, o[8 * cc + 6], o[8 * cc + 7]);
-                }
-              } else {
-                const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                  const int c = 2 * h + g;
-                  const uint32_t spair = scw[c >> 1];
-                  const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
-                  const uint4 w = v[c];
-                  const uint4 q0 = nib8_to_h(w.x, s2), q1 = nib8_to_h(w.y, s2);
-                  const uint4 q2 = nib8_to_h(w.z, s2), q3 = nib8_to_h(w.w, s2);
-                  o[16 * g + 0] = q0.x; o[16 * g + 1] = q0.y; o[16 * g + 2] = q0.z; o[16 * g + 3] = q0.w;
-                  o[16 * g + 4] = q1.x; o[16 * g + 5] = q1.y; o[16 * g + 6] = q1.z; o[16 * g + 7] = q1.w;
-                  o[16 * g + 8] = q2.x; o[16 * g + 9] = q2.y; o[16 * g + 10] = q2.z; o[16 * g + 11] = q2.w;
-                  o[16 * g + 12] = q3.x; o[16 * g + 13] = q3.y; o[16 * g + 14] = q3.z; o[16 * g + 15] = q3.w;
-                }
-              }
-              __syncwarp();  // tcgen05.st is warp-collective
-              tmem_st32(tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCols +
-                            static_cast<uint32_t>(sa) * 32u,
-                        o);
-              tmem_st_wait();
-              tc_fence_before();
-              mbar_arrive(st_full + sa);
-              if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
-              continue;
-            }
-            uint8_t* dst = abuf + sa * kATile;
-            if constexpr (KIND == kQ8) {
-              // raw chunks 4h..4h+3 (16 int8 each) -> fp16 chunks 0..7 of this tile
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                const uint4 w = v[4 * h + cc];
-                uint4 o0, o1;
-                i8x4_to_h(w.x, o0.x, o0.y);
-                i8x4_to_h(w.y, o0.z, o0.w);
-                i8x4_to_h(w.z, o1.x, o1.y);
-                i8x4_to_h(w.w, o1.z, o1.w);
-                *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc)) = o0;
-                *reinterpret_cast<uint4*>(dst + sw128(t, 2 * cc + 1)) = o1;
-              }
-            } else {
-              // raw chunks 2h, 2h+1 (one 32-k group each) -> fp16 chunks 0..7
-              const uint32_t* scw = reinterpret_cast<const uint32_t*>(&sc);
-#pragma unroll
-              for (int g = 0; g < 2; ++g) {
-                const int c = 2 * h + g;
-                const uint32_t spair = scw[c >> 1];
-                const uint32_t s2 = (c & 1) ? __byte_perm(spair, 0, 0x3232) : __byte_perm(spair, 0, 0x1010);
-                const uint4 w = v[c];
-                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 0)) = nib8_to_h(w.x, s2);
-                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 1)) = nib8_to_h(w.y, s2);
-                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 2)) = nib8_to_h(w.z, s2);
-                *reinterpret_cast<uint4*>(dst + sw128(t, 4 * g + 3)) = nib8_to_h(w.w, s2);
-              }
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(st_full + sa);
-            if (++sa == p.n_a) { sa = 0; aph ^= 1u; }
-          }
-        }
-      }
+      const bool ok = dequant_rows(t, 0, (KIND == kQ4 && p.tmem_a) ? 2 : 1);
       // The CTA's last tile: these warps take its odd epilogue chunks, with
       // store boxes staged in the now idle raw-weight ring.
       if (ok && !split && tile0 < p.tiles) {
@@ -938,13 +1034,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           tc_fence_after();
           const uint32_t tacc = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + b * kAccCols;
           uint8_t* sb0 = raw + (warp - 8) * 2 * T::kStageBuf;
-          int nst = 0;
-          for (int c = 1; c < p.BN / 16; c += 2, ++nst) {
-            uint8_t* sbuf = sb0 + (nst & 1) * T::kStageBuf;
-            epilogue_chunk_compute<KIND>(c, tacc, lane, sbuf, rc, sxs);
-            __syncwarp();
-            epilogue_chunk_store<KIND>(c, n0 + (warp & 3) * 32, m0, lane, sbuf, p);
-          }
+          // the last tile's buffer is not reused: nothing to release
+          epilogue_chunks<KIND>(1, 2, p.BN / 16, tacc, lane, sb0, 0, rc, sxs, n0 + (warp & 3) * 32, m0, p,
+                                [] {});
         }
       }
     }
@@ -952,6 +1044,13 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     // ----------------------------------------------------------- epilogue
     // kEpiWarps warps; warp e (0-based) reads TMEM lanes 32*(warp%4).. and
     // takes every (kEpiWarps/4)-th 16-column chunk starting at e/4.
+    if constexpr (KIND == kQ4) {
+      // one tile per CTA (A in tensor memory): these warps have nothing to
+      // do until its accumulator is complete, so they dequantise half of its
+      // K blocks beside warps 8..11 (q4 only: the q8 conversion is cheap
+      // enough for one group, measured no faster with two)
+      if (p.tmem_a) dequant_rows(threadIdx.x - 128, 1, 2);
+    }
     const int e = warp - 4;
     const int nep = T::kEpiWarps * 32;
     const int te = threadIdx.x - 128;
@@ -960,45 +1059,59 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     if (!split) {
       uint8_t* sbuf0 = stage + e * 2 * T::kStageBuf;
+      const float alpha = p.steer ? steer_alpha(p) : 0.0f;
+      // The channel constants and (W8A8) token scales of a tile are loaded
+      // one tile ahead, so their latency hides behind the previous tile's
+      // epilogue; the token scales alternate between two shared buffers.
+      RowRaw rr;
+      if (tile0 < p.tiles) {
+        rr = row_raw<KIND>((tile0 % p.tiles_n) * kTileN + t, p);
+        if constexpr (KIND == kW8A8) {
+          const int m0f = (tile0 / p.tiles_n) * p.BN;
+          if (te < p.BN) sxs[te] = (m0f + te < p.M) ? ld_dep_f32(p.sx + m0f + te) : 0.0f;
+        }
+      }
       int ti = 0, nst = 0;
       for (int tile = tile0; tile < p.tiles; tile += tstep, ++ti) {
         const int b = ti & 1;
         const int n0 = (tile % p.tiles_n) * kTileN;
         const int m0 = (tile / p.tiles_n) * p.BN;
-        const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
-        if constexpr (KIND == kW8A8) {
-          named_bar(1, nep);  // the previous tile's readers of sxs are done
-          for (int j = te; j < p.BN; j += nep) sxs[j] = (m0 + j < p.M) ? __ldg(p.sx + m0 + j) : 0.0f;
-          named_bar(1, nep);
+        const RowConst<KIND> rc = row_const_from<KIND>(rr, n0 + t, p, alpha);
+        const float* sxc = sxs + (ti & 1) * kTileBnMax;
+        const int tnext = tile + tstep;
+        float sx_next = 0.0f;
+        if (tnext < p.tiles) {
+          rr = row_raw<KIND>((tnext % p.tiles_n) * kTileN + t, p);
+          if constexpr (KIND == kW8A8) {
+            const int m0n = (tnext / p.tiles_n) * p.BN;
+            if (te < p.BN && m0n + te < p.M) sx_next = ld_dep_f32(p.sx + m0n + te);
+          }
         }
+        // W8A8: this tile's token scales are in place, and every reader of
+        // the other buffer (the previous tile) is done with it
+        if constexpr (KIND == kW8A8) named_bar(1, nep);
         bool ok = mbar_wait(acc_full + b, (ti >> 1) & 1, abort_flag, 8, wlim);
         ok = __all_sync(0xffffffffu, ok);  // warp-uniform before .sync.aligned TMEM loads
-        if (!ok) continue;  // keep taking part in the named barriers of later tiles
-        if (te == 0 && ti == 0) ARIA_STAMP(6);
-        tc_fence_after();
-        const int nchunk = p.BN / 16;
-        // q8/q4: the dequant warps have no work left during the CTA's last
-        // tile and take its odd chunks (see the end of the dequant role)
-        const int cs = (T::kDequant && tile + tstep >= p.tiles) ? 2 : cstep;
-        if (cgrp >= nchunk) {  // no chunk for this warp: release buffer b at once
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + b);
+        if (ok) {
+          if (te == 0 && ti == 0) ARIA_STAMP(6);
+          tc_fence_after();
+          // q8/q4: the dequant warps have no work left during the CTA's last
+          // tile and take its odd chunks (see the end of the dequant role)
+          const int cs = (T::kDequant && tnext >= p.tiles) ? 2 : cstep;
+          nst = epilogue_chunks<KIND>(cgrp, cs, p.BN / 16, tmem_base + lane_off + b * kAccCols, lane, sbuf0,
+                                      nst, rc, sxc, n0 + (warp & 3) * 32, m0, p, [&] {
+                                        // this warp's last TMEM read of buffer b: the
+                                        // tile after next may reuse it
+                                        tc_fence_before();
+                                        __syncwarp();
+                                        if (lane == 0) mbar_arrive(acc_empty + b);
+                                      });
+          if (te == 0) ARIA_STAMP(7);
         }
-        for (int c = cgrp; c < nchunk; c += cs) {
-          uint8_t* sbuf = sbuf0 + (nst & 1) * T::kStageBuf;
-          const uint32_t tacc = tmem_base + lane_off + b * kAccCols;
-          epilogue_chunk_compute<KIND>(c, tacc, lane, sbuf, rc, sxs);
-          if (c + cs >= nchunk) {
-            // this warp's last TMEM read of buffer b: the tile after next may reuse it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty + b);
-          }
-          epilogue_chunk_store<KIND>(c, n0 + (warp & 3) * 32, m0, lane, sbuf, p);
-          ++nst;
+        // (on a failed wait, keep taking part in the named barriers of later tiles)
+        if constexpr (KIND == kW8A8) {
+          if (tnext < p.tiles && te < p.BN) sxs[((ti + 1) & 1) * kTileBnMax + te] = sx_next;
         }
-        if (te == 0) ARIA_STAMP(7);
       }
     }
   }
@@ -1070,6 +1183,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             }
           }
         }
+        if (threadIdx.x == 0 && ml0 == mb) ARIA_STAMP(20);  // the first partials summed
         uint32_t rare_mask = 0;  // W8A8: elements to redo exactly (bit 4u+k)
 #pragma unroll
         for (int u = 0; u < kRows; ++u) {
@@ -1083,7 +1197,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             const uint32_t a4[4] = {acc[u].x, acc[u].y, acc[u].z, acc[u].w};
             __half h[4];
             if constexpr (KIND == kW8A8) {
-              const float sxm = __ldg(p.sx + m);
+              const float sxm = ld_dep_f32(p.sx + m);
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
                 bool rare;
@@ -1104,6 +1218,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.Y) + o) = *reinterpret_cast<uint2*>(h);
           }
         }
+        if (threadIdx.x == 0 && ml0 == mb) ARIA_STAMP(21);  // their outputs stored
         if constexpr (KIND == kW8A8) {
           // rare elements: round exactly from the summed accumulator (picked
           // from registers by index: no second trip to the peers' shared
@@ -1128,7 +1243,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
             const int32_t a = static_cast<int32_t>(asel);
             const RowConst<kW8A8> rk = row_const<kW8A8>(n + k, p);
             reinterpret_cast<__half*>(p.Y)[static_cast<int64_t>(m) * p.N + n + k] =
-                epi_w8a8(a, __ldg(p.sx + m), rk);
+                epi_w8a8(a, ld_dep_f32(p.sx + m), rk);
           }
         }
       }

@@ -80,12 +80,12 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half*
   for (int i = 0; i < kRowCached; ++i) {
     const int c = threadIdx.x + i * kRowThreads;
     if (c < nchunk) {
-      cache[i] = __ldg(xr + c);
+      cache[i] = ld_dep_v4(xr + c);
       a = fmaxf(a, absmax8(cache[i]));
     }
   }
   for (int c = threadIdx.x + kRowCached * kRowThreads; c < nchunk; c += kRowThreads)
-    a = fmaxf(a, absmax8(__ldg(xr + c)));
+    a = fmaxf(a, absmax8(ld_dep_v4(xr + c)));
 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kRowThreads) row_quant_i8_kernel(const __half*
     if (c < nchunk) qr[c] = quant8_i8(cache[i], s, zero);
   }
   for (int c = threadIdx.x + kRowCached * kRowThreads; c < nchunk; c += kRowThreads)
-    qr[c] = quant8_i8(__ldg(xr + c), s, zero);
+    qr[c] = quant8_i8(ld_dep_v4(xr + c), s, zero);
   if (!early_dependents) publish_packed_stores();
 }
 
@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(256) pack_q4_kernel(const __half* __restrict__
     const int64_t c = base + threadIdx.x;
     const bool live = c < nchunk;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (live) v = __ldg(w4 + c);
+    if (live) v = ld_dep_v4(w4 + c);
     float a = absmax8(v);
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));

@@ -51,13 +51,14 @@ struct SmallParams {
   int rows_base, rows_rem;  // cluster c owns rows_base + (c < rows_rem) rows
   int r_pad;              // 16-aligned maximum rows per cluster
   uint32_t wrow;          // shared-memory bytes per weight row (slice bytes + 16)
-  uint32_t off_sc, off_red, off_part, off_bar;  // shared-memory offsets (weights at 0)
+  uint32_t off_sc, off_red, off_part, off_bar, off_sw;  // shared-memory offsets (weights at 0)
   const uint8_t* W;       // q8 int8 [N,K]; q4 uint8 [N,K/2]; fp16 [N,K]
   const __half* Wsc;      // q4 group scales [N,K/32]
   const float* sw;        // q8 channel scales [N]
   const __half* X;        // [M,K]
   const __half* bias;     // [N] or null
   const float* steer;     // [N] or null
+  int trace_launch;       // trace builds: the launch's index since the trace was cleared
   float alpha;
   const float* alpha_dev;
   __half* Y;              // [M,N]
@@ -138,16 +139,18 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + p.off_bar);
 
   if (tid == 0) {
+    ARIA_STAMP(0);
     mbar_init(bar, 1);
     fence_mbar_init();
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(R) * (slice_bytes + sc_bytes));
   }
   __syncthreads();
-  // ---- all weight bytes of this CTA, before the dependency wait
-  if (warp == 0) {
+  // ---- all weight bytes of this CTA, before the dependency wait: every
+  // thread issues the bulk copies of its share of the rows (one warp issuing
+  // them all serialises the requests)
+  {
     const uint64_t pol = policy_evict_first();  // streamed once
-    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(R) * (slice_bytes + sc_bytes));
-    __syncwarp();
-    for (int r = lane; r < R; r += 32) {
+    for (int r = tid; r < R; r += kSmThreads) {
       const int64_t n = r0 + r;
       bulk_g2s(wsm + r * p.wrow, p.W + n * row_bytes + static_cast<int64_t>(k0) * Tr::kNum / Tr::kDen,
                slice_bytes, bar, pol);
@@ -155,8 +158,15 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
         bulk_g2s(scs + r * (p.kslice / 32), p.Wsc + n * (p.K / 32) + k0 / 32, sc_bytes, bar, pol);
     }
   }
+  // q8: the channel scales of the CTA's rows (part of the pack, like the
+  // weights) into shared memory, also before the wait
+  float* s_sw = reinterpret_cast<float*>(sm + p.off_sw);
+  if constexpr (KIND == kQ8)
+    for (int r = tid; r < R; r += kSmThreads) s_sw[r] = __ldg(p.sw + r0 + r);
+  if (tid == 0) ARIA_STAMP(1);
   pdl_launch_dependents();  // the next launch may start streaming its own weights
   pdl_wait();               // X, the epilogue operands and Y belong to the stream order
+  if (tid == 0) ARIA_STAMP(2);
 
   // ---- this warp's activation chunks into registers: token tb*8 + g4,
   // k values [k0 + 64c + 16q, +16) as two 16-byte vectors
@@ -172,8 +182,8 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
       xb[i][tb] = make_uint4(0u, 0u, 0u, 0u);
       if (c < nch && t < p.M) {
         const uint4* src = reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(t) * p.K + k0 + c * 64 + 16 * q);
-        xa[i][tb] = __ldg(src);
-        xb[i][tb] = __ldg(src + 1);
+        xa[i][tb] = ld_dep_v4(src);
+        xb[i][tb] = ld_dep_v4(src + 1);
       }
     }
   }
@@ -190,6 +200,7 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
       }
     }
   }
+  if (tid == 0) ARIA_STAMP(3);
 
   constexpr int NT = TB * 8;  // tokens per warp tile
   const int groups = (R + 15) >> 4;
@@ -280,23 +291,25 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
       } else if (t < p.M && rl < R) {
         const int n = r0 + rl;
         float y = s;
-        if constexpr (KIND == kQ8) y = __fmul_rn(y, __ldg(p.sw + n));
+        if constexpr (KIND == kQ8) y = __fmul_rn(y, s_sw[rl]);
         if (p.bias) y = __fadd_rn(y, __half2float(p.bias[n]));
         if (p.steer) {
           const float a = p.alpha_dev ? *p.alpha_dev : p.alpha;
-          if (a != 0.0f) y = __fmaf_rn(a, __ldg(p.steer + n), y);
+          if (a != 0.0f) y = __fmaf_rn(a, ld_dep_f32(p.steer + n), y);
         }
         p.Y[static_cast<int64_t>(t) * p.N + n] = __float2half_rn(y);
       }
     }
   }
 
+  if (tid == 0) ARIA_STAMP(4);
   if (p.S > 1) {
     // rank r finishes rows [R*r/S, R*(r+1)/S) of the cluster's range: the S
     // partials through distributed shared memory, added in rank order
     cluster_sync();
     const int rb0 = R * rank / p.S, rb1 = R * (rank + 1) / p.S;
     const int nr = rb1 - rb0;
+    if (tid == 0) ARIA_STAMP(5);
     const uint32_t part_u32 = smem_u32(sm + p.off_part);
     const float a = p.steer ? (p.alpha_dev ? *p.alpha_dev : p.alpha) : 0.0f;
     for (int idx = tid; idx < p.M * nr; idx += kSmThreads) {
@@ -306,13 +319,14 @@ __global__ void __launch_bounds__(kSmThreads, 2) smallm_kernel(const SmallParams
       for (int r = 0; r < p.S; ++r) s += __uint_as_float(ld_dsmem_u32(mapa_shared(part_u32 + off, r)));
       const int n = r0 + rl;
       float y = s;
-      if constexpr (KIND == kQ8) y = __fmul_rn(y, __ldg(p.sw + n));
+      if constexpr (KIND == kQ8) y = __fmul_rn(y, s_sw[rl]);
       if (p.bias) y = __fadd_rn(y, __half2float(p.bias[n]));
-      if (a != 0.0f) y = __fmaf_rn(a, __ldg(p.steer + n), y);
+      if (a != 0.0f) y = __fmaf_rn(a, ld_dep_f32(p.steer + n), y);
       p.Y[static_cast<int64_t>(t) * p.N + n] = __float2half_rn(y);
     }
     cluster_sync();  // no CTA leaves while a peer still reads its partials
   }
+  if (tid == 0) ARIA_STAMP(6);
 }
 
 }  // namespace aria
