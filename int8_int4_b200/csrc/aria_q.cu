@@ -273,6 +273,10 @@ aria_status plan_gemm(int kind, int64_t M, int64_t N, int64_t K, Plan* out) {
   p.off_bar = p.off_sxd + sxd_bytes;
   // the split-K partial tile (BN rows x 512 B) overlays the stage rings
   if (static_cast<uint32_t>(bn) * 512u > p.off_stage) p.splits = splits = 1;
+  // warps 0..3 help with the last tile's epilogue when their store boxes (and
+  // W8A8 token scales) fit in the activation ring
+  const uint64_t helper_bytes = 8ull * kEpiRows * 32 * out_bytes + 4ull * kTileBnMax;
+  p.helpers = static_cast<uint64_t>(nx) * p.x_stage >= helper_bytes ? 1 : 0;
   const uint32_t nbar = 2 * (nr + na) + 6;  // raw, stage, 2 acc_full, 2 acc_empty, mma_drain, acc_last
   const size_t smem = 1024 + p.off_bar + nbar * 8 + 16;
   if (smem > static_cast<size_t>(di.smem_optin)) return fail(ARIA_ERR_UNSUPPORTED, "shared memory plan too large");

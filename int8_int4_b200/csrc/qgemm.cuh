@@ -93,6 +93,9 @@ struct GemmParams {
   // operand) go to tensor memory, columns [kAccCols + 32 s, +32) for stage s,
   // instead of shared memory; the accumulator keeps columns [0, BN)
   int tmem_a;
+  // the CTA's last tile: warps 0..3, done with their roles, take a third of
+  // its epilogue chunks (their store boxes fit in the activation ring)
+  int helpers;
   int trace_launch;       // trace builds: the launch's index since the trace was cleared
   void* Y;                // fp16 [M,N], or int32 [M,N] for kS32 (split-K path)
 };
@@ -635,8 +638,9 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   const int rank = split ? static_cast<int>(cluster_ctarank()) : 0;
   const int tile0 = split ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
   const int tstep = split ? static_cast<int>(gridDim.y) : static_cast<int>(gridDim.x);
-  const int u_begin = static_cast<int>(static_cast<int64_t>(p.units) * rank / p.splits);
-  const int u_end = static_cast<int>(static_cast<int64_t>(p.units) * (rank + 1) / p.splits);
+  // units < 2^26 and rank < 8: the products fit in 32 bits
+  const int u_begin = static_cast<int>(static_cast<unsigned>(p.units) * rank / static_cast<unsigned>(p.splits));
+  const int u_end = static_cast<int>(static_cast<unsigned>(p.units) * (rank + 1) / static_cast<unsigned>(p.splits));
   const int nu = u_end - u_begin;
   const int nkb = nu * T::kKbPerUnit;
 
@@ -663,41 +667,11 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_last + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < p.n_raw; ++i) {
-      mbar_init(raw_full + i, 1);
-      mbar_init(raw_empty + i, (KIND == kQ4 && p.tmem_a) ? 256 : 128);  // the dequant threads
-    }
-    for (int i = 0; i < p.n_a; ++i) {
-      // q8/q4: 128 dequant threads + the X producer; W8A8: the single producer
-      mbar_init(st_full + i, T::kDequant ? 129 : 1);
-      mbar_init(st_empty + i, 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(acc_full + i, 1);
-      mbar_init(acc_empty + i, T::kEpiWarps);
-    }
-    mbar_init(mma_drain, 1);
-    mbar_init(acc_last, 1);
-    *abort_flag = 0;
-    ARIA_STAMP(16);
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmW);
-    prefetch_tmap(&tmX);
-    if constexpr (KIND == kQ4) prefetch_tmap(&tmS);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * kAccCols);
-    tmem_relinquish();
-    if (lane == 0) ARIA_STAMP(18);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (threadIdx.x == 0) ARIA_STAMP(19);
-  const uint32_t tmem_base = *tmem_slot;
+  // ---- prologue. Warp 0 initialises the barriers, one per lane; lane 0
+  // takes the "full" barriers of the first weight loads and issues those
+  // loads at once (they need nothing else), before the CTA-wide barrier that
+  // also waits for the TMEM allocation.
+  //
   // Programmatic dependent launch: this CTA may start while the preceding
   // kernel in the stream drains. Packed weights and their scales are inputs
   // that no kernel of this library writes while a following GEMM can already
@@ -709,43 +683,72 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
   // the preceding kernel to complete.
   int issued_w = 0, issued_x = 0;  // kept for the teardown drain
   int pre = 0;                     // raw units / stages of the first tile issued before the wait
-  if (warp == 0 && tile0 < p.tiles) {
-    const int n0 = (tile0 % p.tiles_n) * kTileN;
-    const uint64_t pol = policy_evict_first();
-    if constexpr (T::kDequant) {
-      pre = nu < p.n_raw ? nu : p.n_raw;
-      if (lane == 0) {
+  if (warp == 0) {
+    if (tile0 < p.tiles) pre = T::kDequant ? (nu < p.n_raw ? nu : p.n_raw) : (nkb < p.n_a ? nkb : p.n_a);
+    uint64_t* pre_full = T::kDequant ? raw_full : st_full;  // arrival count 1 in both rings
+    const int nbar = 2 * (p.n_raw + p.n_a) + 6;
+    if (lane == 0) {
+      for (int i = 0; i < pre; ++i) mbar_init(pre_full + i, 1);
+      *abort_flag = 0;
+    } else {
+      for (int i = lane - 1; i < nbar; i += 31) {
+        uint64_t* bar = bars + i;
+        if (bar >= pre_full && bar < pre_full + pre) continue;  // lane 0's
+        uint32_t cnt = 1;                                         // raw_full, st_empty, acc_full, drain, last
+        if (i >= p.n_raw && i < 2 * p.n_raw)
+          cnt = (KIND == kQ4 && p.tmem_a) ? 256 : 128;            // raw_empty: the dequant threads
+        else if (i >= 2 * p.n_raw && i < 2 * p.n_raw + p.n_a)
+          cnt = T::kDequant ? 129 : 1;                            // st_full: dequant threads + X producer
+        else if (bar == acc_empty || bar == acc_empty + 1)
+          cnt = T::kEpiWarps;
+        mbar_init(bar, cnt);
+      }
+    }
+    fence_mbar_init();
+    if (lane == 0) {
+      ARIA_STAMP(16);
+      prefetch_tmap(&tmW);
+      prefetch_tmap(&tmX);
+      if constexpr (KIND == kQ4) prefetch_tmap(&tmS);
+      if (pre > 0) {
+        const int n0 = (tile0 % p.tiles_n) * kTileN;
+        const uint64_t pol = policy_evict_first();
         for (int i = 0; i < pre; ++i) {
-          const int u = u_begin + i;
-          uint8_t* dst = raw + i * p.raw_stage;
-          if constexpr (KIND == kQ8) {
-            mbar_arrive_expect_tx(raw_full + i, kATile);
-            tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
+          if constexpr (T::kDequant) {
+            const int u = u_begin + i;
+            uint8_t* dst = raw + i * p.raw_stage;
+            if constexpr (KIND == kQ8) {
+              mbar_arrive_expect_tx(raw_full + i, kATile);
+              tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
+            } else {
+              mbar_arrive_expect_tx(raw_full + i, kATile + kQ4ScaleTile);
+              tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
+              tma_load_2d(&tmS, raw_full + i, dst + kATile, u * 8, n0, pol);
+            }
           } else {
-            mbar_arrive_expect_tx(raw_full + i, kATile + kQ4ScaleTile);
-            tma_load_2d(&tmW, raw_full + i, dst, u * 128, n0, pol);
-            tma_load_2d(&tmS, raw_full + i, dst + kATile, u * 8, n0, pol);
+            if (i == 0 && drop0) continue;  // self-test: this stage never fills
+            mbar_arrive_expect_tx(st_full + i, kATile + p.x_stage);
+            tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * T::kWUnitX, n0, pol);
           }
         }
-      }
-    } else {
-      pre = nkb < p.n_a ? nkb : p.n_a;
-      if (lane == 0) {
-        for (int i = 0; i < pre; ++i) {
-          if (i == 0 && drop0) continue;  // self-test: this stage never fills
-          mbar_arrive_expect_tx(st_full + i, kATile + p.x_stage);
-          tma_load_2d(&tmW, st_full + i, abuf + i * kATile, (u_begin + i) * T::kWUnitX, n0, pol);
+        for (int i = pre; i < nu && i < pre + kL2Ahead; ++i) {  // and the next units into L2
+          tma_prefetch_2d(&tmW, (u_begin + i) * T::kWUnitX, n0);
+          if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
         }
       }
     }
     issued_w = pre;
-    if (lane == 0) {  // and the next units into L2
-      for (int i = pre; i < nu && i < pre + kL2Ahead; ++i) {
-        tma_prefetch_2d(&tmW, (u_begin + i) * T::kWUnitX, n0);
-        if constexpr (KIND == kQ4) tma_prefetch_2d(&tmS, (u_begin + i) * 8, n0);
-      }
-    }
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * kAccCols);
+    tmem_relinquish();
+    if (lane == 0) ARIA_STAMP(18);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) ARIA_STAMP(19);
+  const uint32_t tmem_base = *tmem_slot;
   if (threadIdx.x == 0) ARIA_STAMP(1);
   pdl_wait();
   pdl_launch_dependents();
@@ -1035,8 +1038,8 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           const uint32_t tacc = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) + b * kAccCols;
           uint8_t* sb0 = raw + (warp - 8) * 2 * T::kStageBuf;
           // the last tile's buffer is not reused: nothing to release
-          epilogue_chunks<KIND>(1, 2, p.BN / 16, tacc, lane, sb0, 0, rc, sxs, n0 + (warp & 3) * 32, m0, p,
-                                [] {});
+          epilogue_chunks<KIND>(1, p.helpers ? 3 : 2, p.BN / 16, tacc, lane, sb0, 0, rc, sxs,
+                                n0 + (warp & 3) * 32, m0, p, [] {});
         }
       }
     }
@@ -1095,9 +1098,10 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
         if (ok) {
           if (te == 0 && ti == 0) ARIA_STAMP(6);
           tc_fence_after();
-          // q8/q4: the dequant warps have no work left during the CTA's last
-          // tile and take its odd chunks (see the end of the dequant role)
-          const int cs = (T::kDequant && tnext >= p.tiles) ? 2 : cstep;
+          // the CTA's last tile: q8/q4's dequant warps have no work left and
+          // take chunks too (see the end of the dequant role), and so do
+          // warps 0..3 (see below)
+          const int cs = tnext >= p.tiles ? (p.helpers ? 3 : (T::kDequant ? 2 : cstep)) : cstep;
           nst = epilogue_chunks<KIND>(cgrp, cs, p.BN / 16, tmem_base + lane_off + b * kAccCols, lane, sbuf0,
                                       nst, rc, sxc, n0 + (warp & 3) * 32, m0, p, [&] {
                                         // this warp's last TMEM read of buffer b: the
@@ -1113,6 +1117,34 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
           if (tnext < p.tiles && te < p.BN) sxs[((ti + 1) & 1) * kTileBnMax + te] = sx_next;
         }
       }
+    }
+  }
+
+  // ---- the CTA's last tile: warps 0..3 have finished their roles (the
+  // producers issued their last loads, the MMA warp its last commit) and take
+  // every third epilogue chunk from chunk 2. Their store boxes, and for W8A8
+  // their copy of the tile's token scales, sit in the activation ring, idle
+  // once the tile's last MMA has completed (acc_last).
+  if (warp < 4 && p.helpers && !split && tile0 < p.tiles) {
+    const int ti = (p.tiles - tile0 + tstep - 1) / tstep - 1;
+    const int tile = tile0 + ti * tstep;
+    const int n0 = (tile % p.tiles_n) * kTileN;
+    const int m0 = (tile / p.tiles_n) * p.BN;
+    const int t = warp * 32 + lane;  // weight row within the tile == TMEM lane
+    const RowConst<KIND> rc = row_const<KIND>(n0 + t, p);
+    float* hsx = reinterpret_cast<float*>(xbuf + 8 * T::kStageBuf);
+    bool ok = mbar_wait(acc_last, 0, abort_flag, 10, wlim);
+    ok = __all_sync(0xffffffffu, ok);
+    if constexpr (KIND == kW8A8) {
+      if (ok)
+        for (int j = threadIdx.x; j < p.BN; j += 128) hsx[j] = (m0 + j < p.M) ? ld_dep_f32(p.sx + m0 + j) : 0.0f;
+      named_bar(2, 128);
+    }
+    if (ok) {
+      tc_fence_after();
+      epilogue_chunks<KIND>(2, 3, p.BN / 16,
+                            tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + (ti & 1) * kAccCols, lane,
+                            xbuf + warp * 2 * T::kStageBuf, 0, rc, hsx, n0 + warp * 32, m0, p, [] {});
     }
   }
 
