@@ -162,7 +162,7 @@ template <int KIND>
 struct RowConst {
   float sw = 0.0f, bias = 0.0f, alpha = 0.0f, v = 0.0f;  // all formats (W8A8: fp32 copies)
   float av_hi = 0.0f, av_lo = 0.0f;                      // W8A8: alpha*v = av_hi + av_lo exactly
-  float sw_up = 0.0f, sw_dn = 0.0f;                      // W8A8: sw * (1 +- 2^-21), rounded
+  float sw_up = 0.0f, sw_dn = 0.0f;                      // W8A8: sw * (1 +- 2^-22), rounded
   bool has_bias = false, has_steer = false;
 };
 
@@ -202,8 +202,8 @@ __device__ __forceinline__ RowConst<KIND> row_const_from(const RowRaw& r, int n,
   c.has_steer = p.steer != nullptr && alpha != 0.0f;
   if constexpr (KIND == kW8A8) {
     c.sw = r.sw;
-    c.sw_up = __fmul_rn(c.sw, 1.0f + 0x1p-21f);
-    c.sw_dn = __fmul_rn(c.sw, 1.0f - 0x1p-21f);
+    c.sw_up = __fmul_rn(c.sw, 1.0f + 0x1p-22f);
+    c.sw_dn = __fmul_rn(c.sw, 1.0f - 0x1p-22f);
     if (c.has_bias) c.bias = __half2float(__ushort_as_half(r.bias));
     if (c.has_steer) {
       c.alpha = alpha;
@@ -335,15 +335,16 @@ __device__ __noinline__ __half w8a8_fixup(__half h, int32_t acc, float sx, float
 }
 
 // No bias and no steering. With t = fl(fl(acc) * s_x), the two products
-// y_up = fl(t * fl(s_w (1 + 2^-21))) and y_dn = fl(t * fl(s_w (1 - 2^-21)))
-// bracket the reference value E = fl64(fl64(acc * s_x) * s_w): the four fp32
-// roundings on each side (acc, t, the scaled s_w, the product) move a value
-// by at most 4 * 2^-24 relative, less than the 2^-21 margin. Rounding to
-// fp16 is monotonic, so if y_up and y_dn round to the same fp16 value, E
-// does too. One packed conversion rounds both; the halves differ for about
-// 0.1 % of elements (E near an fp16 rounding midpoint), which the caller
-// recomputes with the fp64 sequence. No range check on acc is needed: the
-// int-to-float conversion is one of the four roundings.
+// y_up = fl(t * fl(s_w (1 + 2^-22))) and y_dn = fl(t * fl(s_w (1 - 2^-22)))
+// bracket the reference value E = fl64(fl64(acc * s_x) * s_w): for
+// |acc| < 2^24 (fl(acc) exact) the three fp32 roundings on each side (t, the
+// scaled s_w, the product) move a value by at most 3 * 2^-24 relative, and
+// E differs from the exact product by about 2^-52: less than the 2^-22
+// margin. Rounding to fp16 is monotonic, so if y_up and y_dn round to the
+// same fp16 value, E does too. One packed conversion rounds both; the halves
+// differ for about 0.07 % of elements (E near an fp16 rounding midpoint),
+// which the caller recomputes with the fp64 sequence, as it does for
+// |acc| >= 2^24 (w8a8_acc_big).
 __device__ __forceinline__ uint32_t w8a8_plain_pair(int32_t acc, float sx, float sw_up, float sw_dn) {
   const float t = __fmul_rn(__int2float_rn(acc), sx);
   const float yu = __fmul_rn(t, sw_up);
@@ -354,6 +355,10 @@ __device__ __forceinline__ uint32_t w8a8_plain_pair(int32_t acc, float sx, float
 }
 
 __device__ __forceinline__ bool pair_split(uint32_t pk) { return (pk >> 16) != (pk & 0xFFFFu); }
+
+__device__ __forceinline__ bool w8a8_acc_big(int32_t acc) {
+  return static_cast<uint32_t>(acc) + (1u << 24) >= (1u << 25);  // |acc| >= 2^24
+}
 
 __device__ __forceinline__ __half epi_w8a8(int32_t acc, float sx, const RowConst<kW8A8>& c) {
   W8A8Val v;
@@ -416,7 +421,7 @@ __device__ __forceinline__ void epilogue_chunk_compute(int c, uint32_t tacc, int
         for (int i = 0; i < 16; ++i) {
           const uint32_t pk = w8a8_plain_pair(static_cast<int32_t>(r[i]), sxv[i], rc.sw_up, rc.sw_dn);
           h[i] = __ushort_as_half(static_cast<unsigned short>(pk & 0xFFFFu));
-          rare_mask |= static_cast<uint32_t>(pair_split(pk)) << i;
+          rare_mask |= static_cast<uint32_t>(pair_split(pk) | w8a8_acc_big(static_cast<int32_t>(r[i]))) << i;
         }
       } else {
 #pragma unroll
@@ -1236,7 +1241,7 @@ __global__ void __launch_bounds__(KindTraits<KIND>::kThreads, 1)
                 if (!rc[k].has_bias && !rc[k].has_steer) {
                   const uint32_t pk = w8a8_plain_pair(static_cast<int32_t>(a4[k]), sxm, rc[k].sw_up, rc[k].sw_dn);
                   h[k] = __ushort_as_half(static_cast<unsigned short>(pk & 0xFFFFu));
-                  rare = pair_split(pk);
+                  rare = pair_split(pk) | w8a8_acc_big(static_cast<int32_t>(a4[k]));
                 } else {
                   W8A8Val vv;
                   h[k] = w8a8_round(static_cast<int32_t>(a4[k]), sxm, rc[k], vv, rare);
