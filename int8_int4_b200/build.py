@@ -47,6 +47,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+PROBE_SRC = os.path.join(PKG, "probe", "tc_issue_probe.cu")
+PROBE = os.path.join(PKG, "tc_issue_probe")
+
+
+def build_probe() -> str:
+    """The standalone tcgen05 issue-cost measurement (not part of the library)."""
+    cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+           PROBE_SRC, "-o", PROBE]
+    subprocess.check_call(cmd)
+    return PROBE
+
+
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    if "--probe" in sys.argv:
+        print(build_probe())
+    else:
+        build(force="--force" in sys.argv, verbose="-v" in sys.argv)
+        print(LIB)
